@@ -1,0 +1,359 @@
+/*
+ * bonsai_oracle.c - plain CPU oracle for the weight-only low-bit linear layer.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library.  The CUDA library never
+ * includes, links or calls it, and it includes nothing from the CUDA side.
+ *
+ * What it computes, from the pages:
+ *   - every quantised weight is w = scale_g * t with t in {-1,+1} (binary) or
+ *     {-1,0,+1} (ternary), one FP16 scale shared by a group of 128 weights
+ *     ["Cómo Bonsai Ternary 4B revoluciona la difusión texto-imagen",
+ *     section "Representación y almacenamiento de los pesos ternarios";
+ *     "Introducing 1-bit and Ternary Bonsai Image 4B: Image Generation for
+ *     Local Devices", section "量化数学：1.125 和 1.71 是怎么来的"];
+ *   - the group runs over 128 consecutive weights of one output row, along
+ *     the input dimension K (the reading the rest of the design supports);
+ *   - ternary weights are stored as INT2, two bits per weight ["Cómo
+ *     Bonsai Ternary 4B ...", same section]; binary weights as one bit per
+ *     weight (1 + 16/128 = 1.125 effective bits, "Introducing 1-bit and
+ *     Ternary Bonsai Image 4B ...", same section);
+ *   - out[m,n] = sum_k A[m,k] * w[n,k] with FP16 activations A [M,K] and an
+ *     FP16 result [M,N].
+ *
+ * How: codes are unpacked, each weight is formed as the IEEE product t*s in
+ * double and rounded to FP16, and every output is one double accumulation
+ * over k in ascending order, rounded once to FP16 (round to nearest even).
+ * The FP16 <-> double conversions below are written from the IEEE 754
+ * binary16 definition (1 sign bit, 5 exponent bits with bias 15, 10
+ * fraction bits, subnormals, inf and NaN).
+ *
+ * The bit layout of a packed word is this project's own format; the pages
+ * only fix the number of bits per weight.  It is defined at oracle_pack.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_SHAPE 2
+#define ORACLE_ERR_BAD_CODE 4
+#define ORACLE_ERR_NOMEM 5
+
+#define MODE_BINARY 1
+#define MODE_TERNARY 2
+#define GROUP 128
+
+/* ---------------------------------------------------------------- FP16 -- */
+
+/* binary16 bit pattern -> exact double value. */
+double oracle_half_to_double(uint16_t h) {
+  int negative = (h >> 15) & 1;
+  int expo = (h >> 10) & 0x1f;
+  int frac = h & 0x3ff;
+  double v;
+  if (expo == 0) {
+    v = ldexp((double)frac, -24); /* zero or subnormal: frac * 2^-24 */
+  } else if (expo == 31) {
+    v = frac ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(1024 + frac), expo - 25); /* (1.frac) * 2^(expo-15) */
+  }
+  return negative ? -v : v;
+}
+
+/* double -> nearest binary16, ties to the even significand. */
+uint16_t oracle_double_to_half(double x) {
+  uint16_t sign = signbit(x) ? 0x8000 : 0;
+  if (isnan(x)) return (uint16_t)(sign | 0x7e00);
+  double a = fabs(x);
+  if (isinf(a)) return (uint16_t)(sign | 0x7c00);
+  /* Write a = q * 2^(e-10): normal binades have q in [1024, 2048); below
+   * 2^-14 the spacing is fixed at 2^-24, i.e. e = -14 with q < 1024. */
+  int e;
+  if (a < 0x1p-14) {
+    e = -14;
+  } else {
+    frexp(a, &e); /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;       /* a in [2^e, 2^(e+1)) */
+  }
+  double q = ldexp(a, 10 - e); /* exact: scaling by a power of two */
+  double qi = floor(q);
+  double rest = q - qi; /* exact */
+  if (rest > 0.5 || (rest == 0.5 && fmod(qi, 2.0) != 0.0)) qi += 1.0;
+  if (qi >= 2048.0) { /* rounding carried into the next binade */
+    qi = 1024.0;
+    e += 1;
+  }
+  if (e > 15) return (uint16_t)(sign | 0x7c00); /* overflow -> inf */
+  if (qi < 1024.0) return (uint16_t)(sign | (uint16_t)qi); /* subnormal */
+  return (uint16_t)(sign | ((e + 15) << 10) | ((int)qi - 1024));
+}
+
+void oracle_half_to_double_array(const uint16_t* h, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_half_to_double(h[i]);
+}
+
+void oracle_double_to_half_array(const double* x, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_double_to_half(x[i]);
+}
+
+/* ------------------------------------------------------------- format -- */
+
+/* Weights per 32-bit word. */
+static int per_word(int mode) { return mode == MODE_BINARY ? 32 : 16; }
+
+static int check_mode_shape(int64_t N, int64_t K, int mode) {
+  if (mode != MODE_BINARY && mode != MODE_TERNARY) return ORACLE_ERR_ARG;
+  if (N < 0 || K < 0) return ORACLE_ERR_SHAPE;
+  if (K % GROUP != 0) return ORACLE_ERR_SHAPE;
+  return ORACLE_OK;
+}
+
+/* Bytes of packed weights for an [N,K] matrix (scales not included). */
+int64_t oracle_packed_bytes(int64_t N, int64_t K, int mode) {
+  if (check_mode_shape(N, K, mode) != ORACLE_OK) return -1;
+  return N * (K / per_word(mode)) * 4;
+}
+
+/* Bit position of weight i of a word.
+ *
+ * Both formats pair weights (2p, 2p+1) of a word: weight 2p lives in the
+ * low 16-bit half, weight 2p+1 in the high half, at the same offset.
+ *
+ * binary  (32 weights/word): weight i -> bit 16*(i%2) + 15 - i/2.
+ *         Bit set <=> t = -1, clear <=> t = +1.
+ * ternary (16 weights/word): weight i -> 2-bit field whose low bit is at
+ *         16*(i%2) + 14 - 2*(i/2) (the magnitude, |t|) and whose high bit,
+ *         one above, is the sign.  t=0 -> 00, t=+1 -> 01, t=-1 -> 11;
+ *         the pattern 10 is not a code.
+ * Words run along K: word j of row n holds k = j*per_word .. +per_word-1,
+ * rows of N words each laid out one after the other (row-major [N, K/pw]).
+ */
+static int binary_bit(int i) { return 16 * (i & 1) + 15 - (i >> 1); }
+static int ternary_low_bit(int i) { return 16 * (i & 1) + 14 - 2 * (i >> 1); }
+
+int oracle_pack(const int8_t* codes, int64_t N, int64_t K, int mode, uint32_t* packed) {
+  int rc = check_mode_shape(N, K, mode);
+  if (rc != ORACLE_OK) return rc;
+  const int pw = per_word(mode);
+  const int64_t words = K / pw;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t j = 0; j < words; ++j) {
+      uint32_t word = 0;
+      for (int i = 0; i < pw; ++i) {
+        int t = codes[n * K + j * pw + i];
+        if (mode == MODE_BINARY) {
+          if (t == -1) word |= 1u << binary_bit(i);
+          else if (t != 1) return ORACLE_ERR_BAD_CODE;
+        } else {
+          uint32_t field;
+          if (t == 0) field = 0u;
+          else if (t == 1) field = 1u;
+          else if (t == -1) field = 3u;
+          else return ORACLE_ERR_BAD_CODE;
+          word |= field << ternary_low_bit(i);
+        }
+      }
+      packed[n * words + j] = word;
+    }
+  }
+  return ORACLE_OK;
+}
+
+int oracle_unpack(const uint32_t* packed, int64_t N, int64_t K, int mode, int8_t* codes) {
+  int rc = check_mode_shape(N, K, mode);
+  if (rc != ORACLE_OK) return rc;
+  const int pw = per_word(mode);
+  const int64_t words = K / pw;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t j = 0; j < words; ++j) {
+      uint32_t word = packed[n * words + j];
+      for (int i = 0; i < pw; ++i) {
+        int t;
+        if (mode == MODE_BINARY) {
+          t = ((word >> binary_bit(i)) & 1u) ? -1 : 1;
+        } else {
+          uint32_t field = (word >> ternary_low_bit(i)) & 3u;
+          if (field == 0u) t = 0;
+          else if (field == 1u) t = 1;
+          else if (field == 3u) t = -1;
+          else return ORACLE_ERR_BAD_CODE; /* 10: sign without magnitude */
+        }
+        codes[n * K + j * pw + i] = (int8_t)t;
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* --------------------------------------------------------- dequantise -- */
+
+/* w[n,k] = fp16(t[n,k] * s[n, k/128]); scales are row-major [N, K/128]. */
+static void dequant_row(const int8_t* t_row, const uint16_t* s_row, int64_t K, uint16_t* w_row) {
+  for (int64_t k = 0; k < K; ++k) {
+    double s = oracle_half_to_double(s_row[k / GROUP]);
+    w_row[k] = oracle_double_to_half((double)t_row[k] * s);
+  }
+}
+
+int oracle_dequant(const uint32_t* packed, const uint16_t* scales, int64_t N, int64_t K,
+                   int mode, uint16_t* w) {
+  int rc = check_mode_shape(N, K, mode);
+  if (rc != ORACLE_OK) return rc;
+  int8_t* t = (int8_t*)malloc((size_t)(N * K > 0 ? N * K : 1));
+  if (!t) return ORACLE_ERR_NOMEM;
+  rc = oracle_unpack(packed, N, K, mode, t);
+  if (rc == ORACLE_OK) {
+    for (int64_t n = 0; n < N; ++n) dequant_row(t + n * K, scales + n * (K / GROUP), K, w + n * K);
+  }
+  free(t);
+  return rc;
+}
+
+/* --------------------------------------------------------------- GEMM -- */
+
+typedef struct {
+  const double* a; /* [M,K] activations as doubles */
+  const double* w; /* [N,K] dequantised weights as doubles */
+  int64_t M, N, K;
+  int64_t m_begin, m_end;
+  uint16_t* out;  /* [M,N] fp16, may be NULL */
+  double* acc;    /* [M,N] double sums, may be NULL */
+  double* absacc; /* [M,N] sum of |a*w|, may be NULL */
+} gemm_job;
+
+static void* gemm_rows(void* arg) {
+  gemm_job* j = (gemm_job*)arg;
+  for (int64_t m = j->m_begin; m < j->m_end; ++m) {
+    const double* a = j->a + m * j->K;
+    for (int64_t n = 0; n < j->N; ++n) {
+      const double* w = j->w + n * j->K;
+      double sum = 0.0, sum_abs = 0.0;
+      for (int64_t k = 0; k < j->K; ++k) {
+        double p = a[k] * w[k]; /* exact: two 11-bit significands */
+        sum += p;
+        sum_abs += fabs(p);
+      }
+      if (j->out) j->out[m * j->N + n] = oracle_double_to_half(sum);
+      if (j->acc) j->acc[m * j->N + n] = sum;
+      if (j->absacc) j->absacc[m * j->N + n] = sum_abs;
+    }
+  }
+  return NULL;
+}
+
+/* Dequantise the whole weight matrix into doubles (unpack, then t*s rounded
+ * to fp16 exactly as oracle_dequant, then widened). */
+static int weights_as_double(const uint32_t* packed, const uint16_t* scales, int64_t N, int64_t K,
+                             int mode, double** w_out) {
+  uint16_t* w16 = (uint16_t*)malloc((size_t)(N * K > 0 ? N * K : 1) * sizeof(uint16_t));
+  double* w = (double*)malloc((size_t)(N * K > 0 ? N * K : 1) * sizeof(double));
+  if (!w16 || !w) {
+    free(w16);
+    free(w);
+    return ORACLE_ERR_NOMEM;
+  }
+  int rc = oracle_dequant(packed, scales, N, K, mode, w16);
+  if (rc == ORACLE_OK) oracle_half_to_double_array(w16, N * K, w);
+  free(w16);
+  if (rc != ORACLE_OK) {
+    free(w);
+    return rc;
+  }
+  *w_out = w;
+  return ORACLE_OK;
+}
+
+/* out = A * W^T, one double accumulation per output.  Rows of the output are
+ * split across nthreads worker threads (each output is still one sequential
+ * sum, so the thread count does not change any result). */
+int oracle_gemm(const uint16_t* A, const uint32_t* packed, const uint16_t* scales, int64_t M,
+                int64_t N, int64_t K, int mode, uint16_t* out, double* acc, double* absacc,
+                int nthreads) {
+  int rc = check_mode_shape(N, K, mode);
+  if (rc != ORACLE_OK) return rc;
+  if (M < 0) return ORACLE_ERR_SHAPE;
+  if (nthreads < 1) nthreads = 1;
+  double* w = NULL;
+  rc = weights_as_double(packed, scales, N, K, mode, &w);
+  if (rc != ORACLE_OK) return rc;
+  double* a = (double*)malloc((size_t)(M * K > 0 ? M * K : 1) * sizeof(double));
+  if (!a) {
+    free(w);
+    return ORACLE_ERR_NOMEM;
+  }
+  oracle_half_to_double_array(A, M * K, a);
+
+  if (nthreads > M) nthreads = M > 0 ? (int)M : 1;
+  gemm_job* jobs = (gemm_job*)calloc((size_t)nthreads, sizeof(gemm_job));
+  pthread_t* tids = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+  if (!jobs || !tids) {
+    free(jobs);
+    free(tids);
+    free(a);
+    free(w);
+    return ORACLE_ERR_NOMEM;
+  }
+  for (int i = 0; i < nthreads; ++i) {
+    jobs[i] = (gemm_job){a, w, M, N, K, M * i / nthreads, M * (i + 1) / nthreads, out, acc, absacc};
+  }
+  int started = 0;
+  for (int i = 1; i < nthreads; ++i) {
+    if (pthread_create(&tids[i], NULL, gemm_rows, &jobs[i]) != 0) break;
+    started = i;
+  }
+  gemm_rows(&jobs[0]);
+  for (int i = started + 1; i < nthreads; ++i) gemm_rows(&jobs[i]); /* threads that failed to start */
+  for (int i = 1; i <= started; ++i) pthread_join(tids[i], NULL);
+  free(jobs);
+  free(tids);
+  free(a);
+  free(w);
+  return ORACLE_OK;
+}
+
+/* The same sums for a list of (m, n) output positions, each computed on its
+ * own: only the needed weight rows are unpacked.  Used to check full-size
+ * problems at sampled positions. */
+int oracle_gemm_entries(const uint16_t* A, const uint32_t* packed, const uint16_t* scales,
+                        int64_t M, int64_t N, int64_t K, int mode, const int64_t* ms,
+                        const int64_t* ns, int64_t count, uint16_t* out, double* acc,
+                        double* absacc) {
+  int rc = check_mode_shape(N, K, mode);
+  if (rc != ORACLE_OK) return rc;
+  const int64_t words = K / per_word(mode);
+  int8_t* t = (int8_t*)malloc((size_t)(K > 0 ? K : 1));
+  uint16_t* w16 = (uint16_t*)malloc((size_t)(K > 0 ? K : 1) * sizeof(uint16_t));
+  if (!t || !w16) {
+    free(t);
+    free(w16);
+    return ORACLE_ERR_NOMEM;
+  }
+  rc = ORACLE_OK;
+  for (int64_t i = 0; i < count && rc == ORACLE_OK; ++i) {
+    int64_t m = ms[i], n = ns[i];
+    if (m < 0 || m >= M || n < 0 || n >= N) {
+      rc = ORACLE_ERR_ARG;
+      break;
+    }
+    rc = oracle_unpack(packed + n * words, 1, K, mode, t);
+    if (rc != ORACLE_OK) break;
+    dequant_row(t, scales + n * (K / GROUP), K, w16);
+    double sum = 0.0, sum_abs = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      double p = oracle_half_to_double(A[m * K + k]) * oracle_half_to_double(w16[k]);
+      sum += p;
+      sum_abs += fabs(p);
+    }
+    if (out) out[i] = oracle_double_to_half(sum);
+    if (acc) acc[i] = sum;
+    if (absacc) absacc[i] = sum_abs;
+  }
+  free(t);
+  free(w16);
+  return rc;
+}
