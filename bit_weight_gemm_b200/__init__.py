@@ -1,0 +1,149 @@
+"""Python binding of libbonsai.so, the B200 weight-only low-bit linear layer.
+
+Argument marshalling only: every operation runs in the library's CUDA
+kernels (see include/bonsai.h for the operations, the packed format and the
+error codes).  PyTorch supplies device memory and the current stream.  There
+is no fallback: if the library is missing or the device is not sm_100, calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+BINARY = 1
+TERNARY = 2
+GROUP = 128
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbonsai.so")
+_lock = threading.Lock()
+_lib = None
+
+# Every function the C header declares, with its ctypes signature.
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+SIGNATURES = {
+    "bonsai_packed_bytes": (ctypes.c_size_t, [_I64, _I64, ctypes.c_int]),
+    "bonsai_scale_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "bonsai_pack": (ctypes.c_int, [_P, _I64, _I64, ctypes.c_int, _P, _P]),
+    "bonsai_dequant": (ctypes.c_int, [_P, _P, _I64, _I64, ctypes.c_int, _P, _P]),
+    "bonsai_lowbit_gemm": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P]),
+    "bonsai_get_device_error": (ctypes.c_int, []),
+    "bonsai_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "bonsai_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint64]),
+}
+
+
+class BonsaiError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"{_LIB_PATH} is missing: build it with `python -m bit_weight_gemm_b200.build`")
+            handle = ctypes.CDLL(_LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(handle, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().bonsai_status_string(int(status)).decode()
+
+
+def _mode(mode) -> int:
+    if mode in (BINARY, "binary"):
+        return BINARY
+    if mode in (TERNARY, "ternary"):
+        return TERNARY
+    raise ValueError(f"unknown mode {mode!r}")
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise BonsaiError(what, status)
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> ctypes.c_void_p:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def words_per_row(K: int, mode) -> int:
+    return K // (32 if _mode(mode) == BINARY else 16)
+
+
+def packed_bytes(N: int, K: int, mode) -> int:
+    return int(lib().bonsai_packed_bytes(N, K, _mode(mode)))
+
+
+def scale_bytes(N: int, K: int) -> int:
+    return int(lib().bonsai_scale_bytes(N, K))
+
+
+def pack(codes: torch.Tensor, mode, out: torch.Tensor | None = None) -> torch.Tensor:
+    """int8 codes [N,K] on the device -> packed words (int32 view) [N, K/32] or [N, K/16]."""
+    N, K = codes.shape
+    m = _mode(mode)
+    if out is None:
+        out = torch.empty((N, words_per_row(K, m)), dtype=torch.int32, device=codes.device)
+    _check(lib().bonsai_pack(_dev(codes, "codes", torch.int8), N, K, m, _dev(out, "out", torch.int32), _stream()),
+           "bonsai_pack")
+    return out
+
+
+def dequant(packed: torch.Tensor, scales: torch.Tensor, K: int, mode, out: torch.Tensor | None = None):
+    """-> FP16 [N,K] with w = t*s exactly."""
+    N = packed.shape[0]
+    m = _mode(mode)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    _check(lib().bonsai_dequant(_dev(packed, "packed"), _dev(scales, "scales", torch.float16), N, K, m,
+                                _dev(out, "out", torch.float16), _stream()), "bonsai_dequant")
+    return out
+
+
+def lowbit_gemm(A: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, mode,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """out[M,N] = A[M,K] * (s*t)^T in FP16 with FP32 accumulation."""
+    M, K = A.shape
+    N = packed.shape[0]
+    m = _mode(mode)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib().bonsai_lowbit_gemm(_dev(A, "A", torch.float16), _dev(packed, "packed"),
+                                    _dev(scales, "scales", torch.float16), M, N, K, m,
+                                    _dev(out, "out", torch.float16), _stream()), "bonsai_lowbit_gemm")
+    return out
+
+
+def get_device_error() -> int:
+    return int(lib().bonsai_get_device_error())
+
+
+def selftest_wait_timeout(limit_ns: int) -> int:
+    return int(lib().bonsai_selftest_wait_timeout(int(limit_ns)))

@@ -1,0 +1,251 @@
+// bonsai.cu - the C ABI declared in include/bonsai.h: argument checks, tensor
+// maps, kernel selection and launches.  All arithmetic runs in the kernels of
+// pack_dequant.cuh and gemm_tc.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "bonsai.h"
+#include "gemm_tc.cuh"
+#include "pack_dequant.cuh"
+
+namespace bonsai {
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s: far above any launch's run time
+constexpr unsigned kErrBitTimeout = 1u << 7;             // set by wait_phase()
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_mode(int mode) { return mode == BONSAI_BINARY || mode == BONSAI_TERNARY_INT2; }
+
+// K multiple of 128, sizes non-negative and small enough for 32-bit tile
+// coordinates and 64-bit byte counts.
+int check_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return BONSAI_ERR_SHAPE;
+  if (K % kGroup != 0) return BONSAI_ERR_SHAPE;
+  const int64_t lim = int64_t(1) << 31;
+  if (M >= lim || N >= lim || K >= lim) return BONSAI_ERR_SHAPE;
+  if (N > 0 && K > (int64_t(1) << 62) / N) return BONSAI_ERR_SHAPE;
+  if (M > 0 && K > (int64_t(1) << 62) / M) return BONSAI_ERR_SHAPE;
+  if (M > 0 && N > (int64_t(1) << 62) / M) return BONSAI_ERR_SHAPE;
+  return BONSAI_OK;
+}
+
+// The kernels use tcgen05 and TMA: the device must be sm_100.
+int check_device() {
+  static std::mutex mu;
+  static int cached[64];  // 0 unknown, 1 ok, 2 wrong arch
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BONSAI_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return BONSAI_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return BONSAI_ERR_CUDA;
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cached[dev] == 1 ? BONSAI_OK : BONSAI_ERR_ARCH;
+}
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? BONSAI_OK : BONSAI_ERR_CUDA;
+}
+
+int grid_for(int64_t work_items, int threads) {
+  int64_t blocks = (work_items + threads - 1) / threads;
+  const int64_t cap = 148 * 16;
+  if (blocks > cap) blocks = cap;
+  return blocks < 1 ? 1 : static_cast<int>(blocks);
+}
+
+// ----------------------------------------------------------- tensor maps --
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major 2-D tensor [rows, inner] of `elem` bytes per element, copied in
+// boxes of box_rows x box_inner.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void* base, uint64_t inner,
+              uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem)};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM --
+template <int MODE, int BLOCK_T, int STAGES>
+int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, uint16_t* out,
+                cudaStream_t stream) {
+  using T = GemmTile<MODE, BLOCK_T, STAGES>;
+  auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T, STAGES>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return BONSAI_ERR_CUDA;
+
+  CUtensorMap map_act, map_w;
+  const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
+  if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, BLOCK_T, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BONSAI_ERR_CUDA;
+  if (!make_map(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, words_per_row, N, T::kWordsPerGroup, T::kRows,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BONSAI_ERR_CUDA;
+  const dim3 grid((N + T::kRows - 1) / T::kRows, (M + BLOCK_T - 1) / BLOCK_T);
+  kernel<<<grid, 192, T::kSmemBytes, stream>>>(map_act, map_w, scales, out, M, N, K, kDefaultWaitLimitNs);
+  return launch_status();
+}
+
+template <int MODE>
+int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
+                  uint16_t* out, cudaStream_t stream) {
+  if (M <= 16) return launch_gemm<MODE, 16, 3>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 32) return launch_gemm<MODE, 32, 3>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 64) return launch_gemm<MODE, 64, 3>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 128) return launch_gemm<MODE, 128, 4>(A, packed, scales, M, N, K, out, stream);
+  return launch_gemm<MODE, 256, 3>(A, packed, scales, M, N, K, out, stream);
+}
+
+}  // namespace
+}  // namespace bonsai
+
+using namespace bonsai;
+
+extern "C" {
+
+size_t bonsai_packed_bytes(int64_t N, int64_t K, int mode) {
+  if (!valid_mode(mode) || check_shape(0, N, K) != BONSAI_OK) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) / (mode == BONSAI_BINARY ? 8 : 4);
+}
+
+size_t bonsai_scale_bytes(int64_t N, int64_t K) {
+  if (check_shape(0, N, K) != BONSAI_OK) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K / kGroup) * 2;
+}
+
+int bonsai_pack(const int8_t* codes, int64_t N, int64_t K, int mode, void* packed, void* stream) {
+  if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
+  int rc = check_shape(0, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (N == 0 || K == 0) return BONSAI_OK;
+  if (!codes || !packed) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(packed)) return BONSAI_ERR_ALIGN;
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_pack_bad_code, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return BONSAI_ERR_CUDA;
+  const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
+  const int grid = grid_for(words / 4, 256);
+  if (mode == BONSAI_BINARY)
+    pack_kernel<BONSAI_BINARY><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
+  else
+    pack_kernel<BONSAI_TERNARY_INT2><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
+  if ((rc = launch_status()) != BONSAI_OK) return rc;
+  unsigned bad = 0;
+  if (cudaMemcpyFromSymbolAsync(&bad, g_pack_bad_code, sizeof(bad), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return BONSAI_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BONSAI_ERR_CUDA;
+  return bad ? BONSAI_ERR_BAD_CODE : BONSAI_OK;
+}
+
+int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_t K, int mode, uint16_t* w,
+                   void* stream) {
+  if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
+  int rc = check_shape(0, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (N == 0 || K == 0) return BONSAI_OK;
+  if (!packed || !scales || !w) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(scales) || !aligned16(w)) return BONSAI_ERR_ALIGN;
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
+  const int grid = grid_for(words, 256);
+  if (mode == BONSAI_BINARY)
+    dequant_kernel<BONSAI_BINARY><<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(packed), scales, w, N, K);
+  else
+    dequant_kernel<BONSAI_TERNARY_INT2><<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(packed), scales, w, N, K);
+  return launch_status();
+}
+
+int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int64_t M, int64_t N, int64_t K,
+                       int mode, uint16_t* out, void* stream) {
+  if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
+  int rc = check_shape(M, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (M == 0 || N == 0) return BONSAI_OK;
+  if (!out) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(out)) return BONSAI_ERR_ALIGN;
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 0) {  // empty sum
+    return cudaMemsetAsync(out, 0, static_cast<size_t>(M) * N * 2, st) == cudaSuccess ? BONSAI_OK : BONSAI_ERR_CUDA;
+  }
+  if (!A || !packed || !scales) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(packed) || !aligned16(scales)) return BONSAI_ERR_ALIGN;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  if (mode == BONSAI_BINARY) return dispatch_gemm<BONSAI_BINARY>(A, packed, scales, m, n, k, out, st);
+  return dispatch_gemm<BONSAI_TERNARY_INT2>(A, packed, scales, m, n, k, out, st);
+}
+
+int bonsai_get_device_error(void) {
+  int rc = check_device();
+  if (rc == BONSAI_ERR_CUDA) return rc;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BONSAI_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess) return BONSAI_ERR_CUDA;
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return BONSAI_ERR_CUDA;
+  if (word & kErrBitTimeout) return BONSAI_ERR_TIMEOUT;
+  return word ? BONSAI_ERR_CUDA : BONSAI_OK;
+}
+
+const char* bonsai_status_string(int status) {
+  switch (status) {
+    case BONSAI_OK: return "ok";
+    case BONSAI_ERR_INVALID_ARG: return "invalid argument";
+    case BONSAI_ERR_SHAPE: return "invalid shape";
+    case BONSAI_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case BONSAI_ERR_BAD_CODE: return "code outside the alphabet";
+    case BONSAI_ERR_CUDA: return "CUDA error";
+    case BONSAI_ERR_ARCH: return "device is not sm_100";
+    case BONSAI_ERR_TIMEOUT: return "a bounded wait in a kernel ran out";
+    default: return "unknown status";
+  }
+}
+
+int bonsai_selftest_wait_timeout(uint64_t limit_ns) {
+  int rc = check_device();
+  if (rc != BONSAI_OK) return rc;
+  if ((rc = bonsai_get_device_error()) == BONSAI_ERR_CUDA) return rc;
+  wait_timeout_selftest_kernel<<<1, 32>>>(limit_ns);
+  if (launch_status() != BONSAI_OK) return BONSAI_ERR_CUDA;
+  return bonsai_get_device_error();
+}
+
+}  // extern "C"

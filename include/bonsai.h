@@ -1,0 +1,117 @@
+/*
+ * bonsai.h - C ABI of the B200 (sm_100a) weight-only low-bit linear layer.
+ *
+ * The operation.  A quantised weight is w[n,k] = s[n, k/128] * t[n,k], with
+ * t in {-1,+1} (binary) or {-1,0,+1} (ternary) and one FP16 scale s per
+ * group of 128 consecutive weights along the input dimension K
+ * ("Cómo Bonsai Ternary 4B revoluciona la difusión texto-imagen", section
+ * "Representación y almacenamiento de los pesos ternarios"; "Introducing
+ * 1-bit and Ternary Bonsai Image 4B: Image Generation for Local Devices",
+ * section "量化数学：1.125 和 1.71 是怎么来的").  The layer computes
+ * out[m,n] = sum_k A[m,k] * w[n,k] for FP16 activations A and returns FP16.
+ * Ternary codes are stored as INT2, two bits per weight ("Cómo Bonsai
+ * Ternary 4B ...", same section); binary codes as one bit per weight (1.125
+ * effective bits with the scale, "Introducing 1-bit and Ternary Bonsai
+ * Image 4B ...", same section).
+ *
+ * Packed format (this library's own; the pages fix only the bit counts).
+ * Rows of N, each a run of little-endian uint32 words along K.  Word j of a
+ * row holds weights k = j*P .. j*P+P-1 (P = 32 binary, 16 ternary); local
+ * weight i sits in pair p = i/2 of half h = i%2 (bits 0-15 or 16-31):
+ *   binary : bit 16h + 15 - p; 1 means t = -1, 0 means t = +1;
+ *   ternary: bits 16h + 14 - 2p (magnitude) and 16h + 15 - 2p (sign);
+ *            t = 0 -> 00, t = +1 -> 01, t = -1 -> 11; 10 is not a code.
+ * Scales: FP16 [N, K/128], row-major.  Activations: FP16 [M, K], row-major.
+ * Output: FP16 [M, N], row-major.  FP16 values travel as uint16_t bits.
+ *
+ * Conventions for every call:
+ *   - pointers are caller-owned DEVICE memory, 16-byte aligned, on the
+ *     current CUDA device, unless a parameter says host;
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); work is
+ *     enqueued on it and the call returns before it finishes, unless noted;
+ *   - the library allocates no device memory;
+ *   - the return value is a bonsai_status; on any error nothing is launched
+ *     (argument errors) or the CUDA error is reported as BONSAI_ERR_CUDA;
+ *   - shapes: M >= 0, N >= 0, K >= 0 with K a multiple of 128 (no partial
+ *     groups); zero-sized problems are valid no-ops.
+ */
+#ifndef BONSAI_H_
+#define BONSAI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BONSAI_BINARY = 1,       /* t in {-1,+1}, 1 bit per weight */
+  BONSAI_TERNARY_INT2 = 2  /* t in {-1,0,+1}, 2 bits per weight */
+} bonsai_mode;
+
+typedef enum {
+  BONSAI_OK = 0,
+  BONSAI_ERR_INVALID_ARG = 1, /* unknown mode, null pointer with a non-empty shape */
+  BONSAI_ERR_SHAPE = 2,       /* negative size, K not a multiple of 128, size overflow */
+  BONSAI_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  BONSAI_ERR_BAD_CODE = 4,    /* bonsai_pack met a code outside the alphabet */
+  BONSAI_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+  BONSAI_ERR_ARCH = 6,        /* the current device is not sm_100 */
+  BONSAI_ERR_TIMEOUT = 7      /* a kernel gave up a bounded wait (see bonsai_get_device_error) */
+} bonsai_status;
+
+/* Bytes of packed weights for an [N,K] weight: N*K/8 (binary) or N*K/4
+ * (ternary).  Returns 0 for an invalid mode or shape. */
+size_t bonsai_packed_bytes(int64_t N, int64_t K, int mode);
+
+/* Bytes of the FP16 scales for an [N,K] weight: 2*N*K/128. */
+size_t bonsai_scale_bytes(int64_t N, int64_t K);
+
+/* Pack weight codes.  codes: int8 [N,K] with every value in the mode's
+ * alphabet; packed: bonsai_packed_bytes(N,K,mode) bytes, written in the
+ * format above.  This call is offline (once per weight): it synchronises
+ * `stream` before returning so that it can report BONSAI_ERR_BAD_CODE when a
+ * code is outside the alphabet (packed is then unspecified).  Concurrent
+ * bonsai_pack calls on different streams share the flag that reports it. */
+int bonsai_pack(const int8_t* codes, int64_t N, int64_t K, int mode, void* packed, void* stream);
+
+/* Exact dequantisation: w[n,k] = fp16(t[n,k] * s[n,k/128]), the IEEE
+ * product (bit-exact: +-s, +-0, or NaN for 0*inf and NaN scales).
+ * packed: as written by bonsai_pack; scales: FP16 [N,K/128]; w: FP16 [N,K].
+ * Meant for testing and for callers that want a dense copy. */
+int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_t K, int mode,
+                   uint16_t* w, void* stream);
+
+/* The fused low-bit GEMM: out[m,n] = fp16( sum_k A[m,k] * w[n,k] ).
+ * A: FP16 [M,K]; packed/scales: as above for an [N,K] weight; out: FP16
+ * [M,N].  Products are formed exactly and summed in FP32 on the tensor
+ * cores, then rounded once to FP16 (nearest even).  Scales must be finite
+ * with |s| < 32768 for ternary weights (the kernel forms 2*s*t in FP16);
+ * outside that range the result is unspecified.  out must not overlap A,
+ * packed or scales.  A packed field with the pattern 10 (not a ternary
+ * code) contributes zero. */
+int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int64_t M,
+                       int64_t N, int64_t K, int mode, uint16_t* out, void* stream);
+
+/* Reads and clears the device-side error word of the current device: 0 if
+ * no kernel reported a problem since the last call, else a bonsai_status
+ * (BONSAI_ERR_TIMEOUT when a bounded wait inside a kernel ran out; the
+ * kernel then returned early and its output is unspecified).  Synchronises
+ * the device. */
+int bonsai_get_device_error(void);
+
+/* Human-readable name of a status code (static string). */
+const char* bonsai_status_string(int status);
+
+/* Self-test of the bounded-wait path: launches one kernel that waits on an
+ * mbarrier nobody arrives at, with a limit of `limit_ns` nanoseconds, and
+ * returns what the kernel recorded: BONSAI_ERR_TIMEOUT when the wait gave up
+ * as designed.  Clears the device error word before and after. */
+int bonsai_selftest_wait_timeout(uint64_t limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BONSAI_H_ */

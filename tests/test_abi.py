@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/bonsai.h declares, and rejects bad arguments before
+touching a device.  Also checks that the CUDA side and the oracle stay
+independent."""
+import os
+import re
+import subprocess
+
+import pytest
+
+import bit_weight_gemm_b200 as bw
+from bit_weight_gemm_b200 import build as bw_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bonsai.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    bw_build.build()
+    return bw.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bonsai_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ["bonsai_pack", "bonsai_dequant", "bonsai_lowbit_gemm", "bonsai_get_device_error",
+                     "bonsai_status_string", "bonsai_packed_bytes", "bonsai_scale_bytes"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", bw.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (bonsai_\w+)", out))
+    declared = set(declared_functions())
+    assert declared <= exported, declared - exported
+    assert declared == set(bw.SIGNATURES), "binding and header disagree"
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_library_does_not_need_libcuda(lib):
+    out = subprocess.run(["readelf", "-d", bw.library_path()], capture_output=True, text=True, check=True).stdout
+    assert "libcuda.so" not in out  # driver calls go through the runtime's entry-point lookup
+
+
+def test_library_is_built_for_sm100a(lib):
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", bw.library_path()], capture_output=True,
+                         text=True).stdout
+    assert "sm_100a" in out
+
+
+def test_sizes(lib):
+    assert bw.packed_bytes(3072, 9216, "ternary") == 3072 * 9216 // 4
+    assert bw.packed_bytes(3072, 9216, "binary") == 3072 * 9216 // 8
+    assert bw.scale_bytes(3072, 9216) == 3072 * 72 * 2
+    assert bw.packed_bytes(8, 100, "ternary") == 0  # partial group
+    assert lib.bonsai_packed_bytes(8, 128, 3) == 0  # unknown mode
+    assert lib.bonsai_packed_bytes(-1, 128, 2) == 0
+
+
+def test_argument_errors_before_any_device_work(lib):
+    P = None
+    assert lib.bonsai_pack(P, 4, 128, 3, P, P) == 1  # mode
+    assert lib.bonsai_pack(P, 4, 100, 2, P, P) == 2  # K % 128
+    assert lib.bonsai_pack(P, -4, 128, 2, P, P) == 2
+    assert lib.bonsai_pack(P, 0, 128, 2, P, P) == 0  # empty: no-op
+    assert lib.bonsai_pack(P, 4, 128, 2, P, P) == 1  # null with data
+    assert lib.bonsai_pack(8, 4, 128, 2, 16, P) == 3  # misaligned
+    assert lib.bonsai_dequant(P, P, 4, 130, 1, P, P) == 2
+    assert lib.bonsai_dequant(16, 16, 4, 128, 1, 24, P) == 3
+    assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 128, 0, P, P) == 1
+    assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 129, 2, P, P) == 2
+    assert lib.bonsai_lowbit_gemm(P, P, P, 0, 4, 128, 2, P, P) == 0
+    assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 128, 2, P, P) == 1
+    assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 128, 2, 8, P) == 3
+    assert lib.bonsai_lowbit_gemm(P, P, P, 1 << 31, 4, 128, 2, 16, P) == 2
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert bw.status_string(s) != "unknown status"
+    assert bw.status_string(99) == "unknown status"
+
+
+def _imports(path):
+    text = open(path, encoding="utf-8").read()
+    return set(re.findall(r"^\s*(?:from|import)\s+([\w\.]+)", text, flags=re.M))
+
+
+def _includes(path):
+    return set(re.findall(r'#include\s+[<"]([^>"]+)[>"]', open(path, encoding="utf-8").read()))
+
+
+def test_cuda_path_and_oracle_share_nothing():
+    pkg = os.path.join(ROOT, "bit_weight_gemm_b200")
+    orc = os.path.join(ROOT, "oracle")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            p = os.path.join(dirpath, f)
+            if f.endswith(".py"):
+                assert not any(i.split(".")[0] in ("oracle", "workloads") for i in _imports(p)), p
+            if f.endswith((".cu", ".cuh", ".h")):
+                assert not any("oracle" in i for i in _includes(p)), p
+    for f in os.listdir(orc):
+        p = os.path.join(orc, f)
+        if f.endswith(".py"):
+            assert not any(i.split(".")[0] in ("bit_weight_gemm_b200", "workloads") for i in _imports(p)), p
+        if f.endswith(".c"):
+            assert all(i in ("math.h", "pthread.h", "stdint.h", "stdlib.h", "string.h") for i in _includes(p)), p

@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA library, called through its C ABI, against the CPU
+oracle on the same seeded inputs.
+
+Bars: pack and dequant bit-exact (NaN compared as NaN); GEMM element-wise
+|gpu - oracle| <= 1e-3 * sum_k |a_k w_k| + one FP16 ulp of the oracle value.
+Small and ragged shapes are compared in full; the full-size workloads at the
+positions the oracle computes one by one (random positions plus every tile
+edge and the last row and column).
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_weight_gemm_b200 as bw
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    bw.lib()
+    assert bw.get_device_error() == 0
+    yield
+    assert bw.get_device_error() == 0, "a kernel recorded a device-side error"
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    return t.cuda()
+
+
+def to_u16(t):
+    return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def to_u32(t):
+    return t.cpu().contiguous().numpy().view(np.uint32)
+
+
+def nan_aware_equal(a, b):
+    a = np.asarray(a, np.uint16)
+    b = np.asarray(b, np.uint16)
+    an = np.isnan(a.view(np.float16))
+    bn = np.isnan(b.view(np.float16))
+    return np.where(an | bn, an & bn, a == b)
+
+
+def gpu_inputs(d, oracle_mod):
+    packed_ref = oracle_mod.pack(d["codes"], d["mode"])
+    codes = dev(d["codes"])
+    packed = bw.pack(codes, d["mode"])
+    torch.cuda.synchronize()
+    return packed_ref, packed, dev(d["A"].view(np.int16), torch.float16), dev(d["scales"].view(np.int16), torch.float16)
+
+
+def assert_gemm_close(oracle_mod, got_bits, ref_bits, absacc, label):
+    ok = oracle_mod.within_tolerance(got_bits, ref_bits, absacc, RTOL)
+    if not ok.all():
+        idx = np.argwhere(~ok)[:5]
+        g = oracle_mod.half_bits_to_double(got_bits)
+        r = oracle_mod.half_bits_to_double(ref_bits)
+        details = [(tuple(i), g[tuple(i)], r[tuple(i)], absacc[tuple(i)]) for i in idx]
+        pytest.fail(f"{label}: {int((~ok).sum())} of {ok.size} outside tolerance, e.g. {details}")
+
+
+# ------------------------------------------------------------------ pack
+PACK_SHAPES = [(1, 128), (37, 384), (256, 256), (129, 1152), (1000, 3072)]
+
+
+@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("N,K", PACK_SHAPES)
+def test_pack_bit_exact(oracle_mod, mode, N, K):
+    d = workloads.make(mode=mode, M=1, N=N, K=K, seed=N * 7 + K)
+    ref = oracle_mod.pack(d["codes"], mode)
+    got = bw.pack(dev(d["codes"]), mode)
+    assert np.array_equal(to_u32(got), ref)
+
+
+@pytest.mark.parametrize("mode,bad", [("ternary", 2), ("ternary", -2), ("binary", 0), ("binary", 3)])
+def test_pack_reports_bad_codes(mode, bad):
+    c = np.ones((64, 256), np.int8)
+    c[63, 255] = bad
+    with pytest.raises(bw.BonsaiError) as e:
+        bw.pack(dev(c), mode)
+    assert e.value.status == 4
+    c[63, 255] = 1
+    bw.pack(dev(c), mode)  # the flag was reset by the failing call
+
+
+# --------------------------------------------------------------- dequant
+@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("N,K", PACK_SHAPES)
+def test_dequant_bit_exact(oracle_mod, mode, N, K):
+    d = workloads.make(mode=mode, M=1, N=N, K=K, seed=N * 3 + K)
+    ref_packed, packed, _, scales = gpu_inputs(d, oracle_mod)
+    ref = oracle_mod.dequant(ref_packed, d["scales"], K, mode)
+    got = bw.dequant(packed, scales, K, mode)
+    assert np.all(nan_aware_equal(to_u16(got), ref))
+
+
+@pytest.mark.parametrize("mode", ["binary", "ternary"])
+def test_dequant_every_scale_pattern(oracle_mod, mode):
+    N, K = 65536, 128
+    rng = np.random.default_rng(12)
+    c = workloads.codes(rng, N, K, mode)
+    s = np.arange(N, dtype=np.uint32).astype(np.uint16)[:, None]
+    ref_packed = oracle_mod.pack(c, mode)
+    ref = oracle_mod.dequant(ref_packed, s, K, mode)
+    got = bw.dequant(dev(ref_packed.view(np.int32)), dev(s.view(np.int16), torch.float16), K, mode)
+    assert np.all(nan_aware_equal(to_u16(got), ref))
+
+
+# ------------------------------------------------------------------ GEMM
+SMALL_SHAPES = [
+    (1, 8, 128), (5, 130, 256), (16, 128, 128), (17, 200, 384), (33, 256, 640), (64, 384, 256),
+    (65, 129, 1152), (128, 256, 512), (129, 300, 256), (255, 128, 384), (256, 512, 256), (300, 384, 512),
+    (513, 136, 768),
+]
+
+
+def _gemm_case(oracle_mod, mode, M, N, K, seed):
+    d = workloads.make(mode=mode, M=M, N=N, K=K, seed=seed)
+    ref_packed, packed, A, scales = gpu_inputs(d, oracle_mod)
+    out = bw.lowbit_gemm(A, packed, scales, mode)
+    torch.cuda.synchronize()
+    ref, _, absacc = oracle_mod.gemm(d["A"], ref_packed, d["scales"], K, mode)
+    return to_u16(out), ref, absacc
+
+
+def test_gemm_ternary_tiny_config(oracle_mod):
+    p = workloads.TERNARY_TINY
+    got, ref, absacc = _gemm_case(oracle_mod, p.mode, p.M, p.N, p.K, p.seed)
+    assert_gemm_close(oracle_mod, got, ref, absacc, p.name)
+
+
+@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("M,N,K", SMALL_SHAPES)
+def test_gemm_ragged_shapes(oracle_mod, mode, M, N, K):
+    got, ref, absacc = _gemm_case(oracle_mod, mode, M, N, K, seed=M * 31 + N * 7 + K)
+    assert_gemm_close(oracle_mod, got, ref, absacc, f"{mode} {M}x{N}x{K}")
+
+
+def test_gemm_binary_512_linear_full(oracle_mod):
+    p = workloads.BINARY_512_LINEAR
+    got, ref, absacc = _gemm_case(oracle_mod, p.mode, p.M, p.N, p.K, p.seed)
+    assert_gemm_close(oracle_mod, got, ref, absacc, p.name)
+
+
+def _sample_positions(M, N, block_t, count, seed):
+    rng = np.random.default_rng(seed)
+    ms = list(rng.integers(0, M, count))
+    ns = list(rng.integers(0, N, count))
+    edges_m = sorted({0, M - 1} | {x for b in range(block_t, M, block_t) for x in (b - 1, b)})
+    edges_n = sorted({0, N - 1} | {x for b in range(128, N, 128) for x in (b - 1, b)})
+    for m in edges_m[:64]:
+        ms += [m] * 8
+        ns += list(rng.integers(0, N, 8))
+    for n in edges_n[:160]:
+        ms += list(rng.integers(0, M, 4))
+        ns += [n] * 4
+    return np.array(ms, np.int64), np.array(ns, np.int64)
+
+
+FULL = [workloads.TERNARY_MLP_UP_4608, workloads.TERNARY_MLP_DOWN_4608, workloads.TERNARY_QKV_4608,
+        workloads.TERNARY_MLP_DOWN_16, workloads.TERNARY_QKV_16]
+
+
+@pytest.mark.parametrize("problem", FULL, ids=[p.name for p in FULL])
+def test_gemm_full_size_sampled(oracle_mod, problem):
+    d = workloads.make(problem)
+    ref_packed, packed, A, scales = gpu_inputs(d, oracle_mod)
+    out = bw.lowbit_gemm(A, packed, scales, problem.mode)
+    got = to_u16(out)
+    ms, ns = _sample_positions(problem.M, problem.N, 256 if problem.M > 128 else 16, 3000, problem.seed)
+    ref, _, absacc = oracle_mod.gemm_entries(d["A"], ref_packed, d["scales"], problem.K, problem.mode, ms, ns)
+    assert_gemm_close(oracle_mod, got[ms, ns], ref, absacc, problem.name)
+    # every output written: no NaN/inf (inputs are bounded) and no untouched rows
+    assert np.isfinite(got.view(np.float16)).all()
+
+
+# ------------------------------------------------------------ invariants
+@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("M", [16, 200])
+def test_gemm_sign_symmetry_bitwise(mode, M):
+    d = workloads.make(mode=mode, M=M, N=256, K=512, seed=M + 5)
+    A = dev(d["A"].view(np.int16), torch.float16)
+    s = dev(d["scales"].view(np.int16), torch.float16)
+    pos = bw.lowbit_gemm(A, bw.pack(dev(d["codes"]), mode), s, mode)
+    neg = bw.lowbit_gemm(A, bw.pack(dev(-d["codes"]), mode), s, mode)
+    assert torch.equal(neg, -pos)
+
+
+@pytest.mark.parametrize("mode", ["binary", "ternary"])
+def test_gemm_power_of_two_scaling_bitwise(mode):
+    d = workloads.make(mode=mode, M=100, N=384, K=384, seed=77)
+    A = dev(d["A"].view(np.int16), torch.float16)
+    s = dev(d["scales"].view(np.int16), torch.float16)
+    p = bw.pack(dev(d["codes"]), mode)
+    one = bw.lowbit_gemm(A, p, s, mode)
+    two = bw.lowbit_gemm(A * 2, p, s, mode)
+    assert torch.equal(two, one * 2)
+
+
+@pytest.mark.parametrize("mode", ["binary", "ternary"])
+def test_gemm_all_ones_closed_form(oracle_mod, mode):
+    N, K = 256, 1024
+    rng = np.random.default_rng(99)
+    c = workloads.codes(rng, N, K, mode)
+    s = workloads.scales(rng, N, K)
+    want = (c.reshape(N, K // 128, 128).astype(np.float64).sum(axis=2) *
+            s.view(np.float16).astype(np.float64)).sum(axis=1)
+    A = torch.ones((48, K), dtype=torch.float16, device="cuda")
+    out = bw.lowbit_gemm(A, bw.pack(dev(c), mode), dev(s.view(np.int16), torch.float16), mode)
+    got = out.double().cpu().numpy()
+    absw = (np.abs(c).reshape(N, K // 128, 128).sum(axis=2) * s.view(np.float16).astype(np.float64)).sum(axis=1)
+    ref_bits = oracle_mod.double_to_half_bits(want)
+    tol = RTOL * absw + oracle_mod.ulp16(ref_bits)
+    assert np.all(np.abs(got - want[None, :]) <= tol[None, :] + np.abs(want)[None, :] * 2.0 ** -11)
+
+
+def test_gemm_rows_independent():
+    d = workloads.make(mode="ternary", M=64, N=256, K=512, seed=3)
+    A = dev(d["A"].view(np.int16), torch.float16)
+    s = dev(d["scales"].view(np.int16), torch.float16)
+    p = bw.pack(dev(d["codes"]), "ternary")
+    base = bw.lowbit_gemm(A, p, s, "ternary")
+    A2 = A.clone()
+    A2[1:] = torch.randn_like(A2[1:])
+    assert torch.equal(bw.lowbit_gemm(A2, p, s, "ternary")[0], base[0])
+
+
+def test_gemm_matches_dequant_then_torch_matmul():
+    """Secondary cross-check (not the oracle): GPU dequant -> fp32 matmul."""
+    d = workloads.make(mode="ternary", M=300, N=512, K=1024, seed=8)
+    A = dev(d["A"].view(np.int16), torch.float16)
+    s = dev(d["scales"].view(np.int16), torch.float16)
+    p = bw.pack(dev(d["codes"]), "ternary")
+    W = bw.dequant(p, s, 1024, "ternary")
+    ref = A.float() @ W.float().T
+    got = bw.lowbit_gemm(A, p, s, "ternary").float()
+    bound = 1e-3 * (A.float().abs() @ W.float().abs().T) + ref.abs() * 2.0 ** -10 + 2.0 ** -24
+    assert bool(((got - ref).abs() <= bound).all())
+
+
+# ------------------------------------------------------------ edge cases
+def test_gemm_empty_shapes():
+    A = torch.zeros((0, 128), dtype=torch.float16, device="cuda")
+    p = torch.zeros((8, 8), dtype=torch.int32, device="cuda")
+    s = torch.zeros((8, 1), dtype=torch.float16, device="cuda")
+    assert bw.lowbit_gemm(A, p, s, "ternary").shape == (0, 8)
+    A = torch.ones((4, 0), dtype=torch.float16, device="cuda")
+    out = bw.lowbit_gemm(A, torch.zeros((8, 0), dtype=torch.int32, device="cuda"),
+                         torch.zeros((8, 0), dtype=torch.float16, device="cuda"), "ternary",
+                         out=torch.full((4, 8), 7.0, dtype=torch.float16, device="cuda"))
+    assert torch.equal(out, torch.zeros_like(out))
+
+
+def test_gemm_zero_codes_and_zero_scales():
+    K = 384
+    A = torch.randn((40, K), dtype=torch.float16, device="cuda")
+    s = torch.rand((200, K // 128), dtype=torch.float16, device="cuda")
+    z = bw.pack(torch.zeros((200, K), dtype=torch.int8, device="cuda"), "ternary")
+    assert not bw.lowbit_gemm(A, z, s, "ternary").any()
+    c = bw.pack(torch.ones((200, K), dtype=torch.int8, device="cuda"), "binary")
+    assert not bw.lowbit_gemm(A, c, torch.zeros_like(s), "binary").any()
+
+
+def test_misaligned_pointer_rejected():
+    buf = torch.zeros(4 * 128 + 8, dtype=torch.float16, device="cuda")
+    A = buf[1:1 + 4 * 128].view(4, 128)
+    p = torch.zeros((8, 8), dtype=torch.int32, device="cuda")
+    s = torch.zeros((8, 1), dtype=torch.float16, device="cuda")
+    with pytest.raises(bw.BonsaiError) as e:
+        bw.lowbit_gemm(A, p, s, "ternary")
+    assert e.value.status == 3
+
+
+def test_bounded_wait_gives_up_and_reports():
+    assert bw.selftest_wait_timeout(2_000_000) == 7  # 2 ms, nobody arrives: BONSAI_ERR_TIMEOUT
+    assert bw.get_device_error() == 0
+    d = workloads.make(workloads.TERNARY_TINY)
+    out = bw.lowbit_gemm(dev(d["A"].view(np.int16), torch.float16), bw.pack(dev(d["codes"]), "ternary"),
+                         dev(d["scales"].view(np.int16), torch.float16), "ternary")
+    torch.cuda.synchronize()
+    assert out.isfinite().all()
