@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the fused low-bit GEMM on B200.
+
+Headline: ternary low-bit W.A GEMM at M=4608 tokens (1024x1024 image + 512
+text tokens), K=3072, N=9216 (MLP-up of a hidden-3072 MMDiT block), in
+FP16-equivalent TFLOP/s (2*M*N*K per launch) and as a fraction of the
+tensor-core roofline.  A step is one call of bonsai_lowbit_gemm: TMA staging,
+unpack + scale, tcgen05 MMA and the FP16 epilogue.  The weights are packed
+once before timing (packing is an offline, once-per-weight step); the
+small-M line reports the bandwidth-bound regime (M=16, ternary MLP-down
+3072x9216) in GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bonsai|reference]
+
+Under torchrun each rank runs an independent replica of the same per-GPU
+workload (weak scaling, no collective on the data path); the timed region
+is bracketed by barriers and the slowest rank's time is reported.
+`--impl reference` times the CPU oracle on bounded samples of the same
+workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+WORKLOAD = workloads.TERNARY_MLP_UP_4608
+SMALL = workloads.TERNARY_MLP_DOWN_16
+METRIC = "low-bit W.A GEMM TFLOP/s (M=4608,K=3072,N=9216 ternary)"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["bonsai", "reference"], default="bonsai")
+    ap.add_argument("--sets", type=int, default=4, help="rotating input sets (their sum exceeds L2)")
+    ap.add_argument("--no-extras", action="store_true", help="skip small-M, e2e, CPU baseline, clocks")
+    ap.add_argument("--small-only", action="store_true", help="time only the M=16 workload (for profiling)")
+    return ap.parse_args()
+
+
+def flops(p) -> int:
+    return 2 * p.M * p.N * p.K
+
+
+def algorithmic_bytes(p) -> int:
+    """Packed weights + FP16 scales + FP16 activations in + FP16 output."""
+    wbytes = p.N * p.K // (8 if p.mode == "binary" else 4)
+    return wbytes + 2 * p.N * (p.K // 128) + 2 * p.M * p.K + 2 * p.M * p.N
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_weight_gemm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- helpers
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_baseline(problem, budget_s: float = 12.0, rows: int = 64):
+    """The oracle, as it stands, on a bounded sample of the workload: `rows`
+    token rows against as many weight rows as fit the time budget."""
+    import oracle
+
+    d = workloads.make(problem)
+    packed = oracle.pack(d["codes"], problem.mode)
+    threads = oracle.default_threads()
+    # calibrate on a small block, then size the sample to the budget
+    n_cal = 256
+    t0 = time.perf_counter()
+    oracle.gemm(d["A"][:rows], packed[:n_cal], d["scales"][:n_cal], problem.K, problem.mode, threads=threads,
+                want_acc=False)
+    t_cal = time.perf_counter() - t0
+    n = int(min(problem.N, max(n_cal, n_cal * budget_s / max(t_cal, 1e-3))))
+    t0 = time.perf_counter()
+    oracle.gemm(d["A"][:rows], packed[:n], d["scales"][:n], problem.K, problem.mode, threads=threads,
+                want_acc=False)
+    dt = time.perf_counter() - t0
+    value = 2 * rows * n * problem.K / dt / 1e12
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} token rows x {n} weight rows x K={problem.K} of {problem.name} "
+                      f"({dt:.1f} s, C oracle, double accumulation, {threads} threads)"}
+
+
+# ------------------------------------------------------------- reference
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    import oracle
+
+    p = WORKLOAD
+    d = workloads.make(p)
+    packed = oracle.pack(d["codes"], p.mode)
+    threads = oracle.default_threads()
+    rows, n_blk = 16, 128
+    # size each step so that warm-up + timed steps end within ~2.5 minutes
+    t0 = time.perf_counter()
+    oracle.gemm(d["A"][:rows], packed[:n_blk], d["scales"][:n_blk], p.K, p.mode, threads=threads, want_acc=False)
+    t_blk = time.perf_counter() - t0
+    per_step = 150.0 / max(1, args.steps + args.warmup)
+    n_blk = int(max(8, min(p.N, n_blk * per_step / max(t_blk, 1e-4))))
+    n_tiles = max(1, p.N // n_blk)
+
+    def step(i):
+        m0 = (i * rows) % (p.M - rows)
+        n0 = (i % n_tiles) * n_blk
+        oracle.gemm(d["A"][m0:m0 + rows], packed[n0:n0 + n_blk], d["scales"][n0:n0 + n_blk], p.K, p.mode,
+                    threads=threads, want_acc=False)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = 2 * rows * n_blk * p.K * args.steps / dt / 1e12
+    sample = (f"each step: {rows} token rows x {n_blk} weight rows x K={p.K} of {p.name}, "
+              f"C oracle with double accumulation on {threads} threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "mode": p.mode, "group": 128},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- bonsai
+def make_sets(problem, count, torch, bw, distinct_weights=True):
+    """`count` input sets on the device.  Each set has its own buffers; with
+    distinct_weights the codes differ too (seed + i)."""
+    sets = []
+    base = None
+    for i in range(count):
+        if distinct_weights or base is None:
+            d = workloads.make(mode=problem.mode, M=problem.M, N=problem.N, K=problem.K, seed=problem.seed + 100 * i)
+            A = torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).cuda()
+            s = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+            packed = bw.pack(torch.from_numpy(d["codes"]).cuda(), problem.mode)
+            base = (A, packed, s)
+        else:
+            A, packed, s = (t.clone() for t in base)
+        out = torch.empty((problem.M, problem.N), dtype=torch.float16, device="cuda")
+        sets.append((A, packed, s, out))
+    torch.cuda.synchronize()
+    return sets
+
+
+def time_launches(torch, bw, problem, sets, steps, warmup, dist=None):
+    """Device time of `steps` back-to-back launches (CUDA events on the
+    launching stream), rotating over the input sets."""
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        A, p, s, o = sets[i % len(sets)]
+        bw.lowbit_gemm(A, p, s, problem.mode, out=o)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        A, p, s, o = sets[i % len(sets)]
+        bw.lowbit_gemm(A, p, s, problem.mode, out=o)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return start.elapsed_time(end) / 1e3  # seconds
+
+
+def run_bonsai(args):
+    import torch
+
+    world, rank, local = dist_setup(args)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+
+    import bit_weight_gemm_b200 as bw
+
+    bw.lib()
+    peaks, peaks_kind = load_peaks()
+    p = WORKLOAD
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras and not args.small_only:
+        cpu = cpu_baseline(p)  # before the first GPU work: the oracle runs threads, no fork
+
+    result = {}
+    if not args.small_only:
+        sets = make_sets(p, args.sets, torch, bw)
+        sampler = ClockSampler(local) if not args.no_extras else None
+        if sampler:
+            sampler.start()
+        secs = time_launches(torch, bw, p, sets, args.steps, args.warmup, dist)
+        clocks = sampler.stop() if sampler else None
+        t = torch.tensor([secs], dtype=torch.float64, device="cuda")
+        if dist is not None:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        secs_max = float(t.item())
+        per_launch = secs_max / args.steps
+        value = flops(p) * args.steps * world / secs_max / 1e12
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        achieved = flops(p) / per_launch / 1e12
+        result.update(value=value, ms_per_step=per_launch * 1e3, clocks=clocks, achieved=achieved, peak=peak)
+        del sets
+
+        e2e = None
+        if not args.no_extras:
+            e2e = time_e2e(torch, bw, p, min(args.steps, 50), 3, dist)
+        result["e2e"] = e2e
+
+    small = None
+    if not args.no_extras or args.small_only:
+        small = time_small(torch, bw, SMALL, args, dist, peaks, peaks_kind)
+
+    if dist is not None:
+        dist.barrier()
+    if rank == 0:
+        if args.small_only:
+            print(json.dumps({"small_m": small}), flush=True)
+        else:
+            traffic = ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}")
+            line = {
+                "metric": METRIC, "value": result["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": result["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+                "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "mode": p.mode, "group": 128,
+                           "parallelism": f"replicas{world}",
+                           "l2": f"{args.sets} rotating input sets, {args.sets * (algorithmic_bytes(p)) / 1e6:.0f} MB "
+                                 f"total > 126 MB L2"},
+                "roofline": {"bound": "tensor", "achieved": result["achieved"], "peak": result["peak"],
+                             "unit": "TFLOP/s", "frac": result["achieved"] / result["peak"],
+                             "traffic": traffic, "peak_source": f"{peaks_kind} bf16 dense (fp16 same nominal rate)"},
+                "gpu_launches": args.steps,
+                "clocks": result["clocks"],
+                "e2e": result["e2e"],
+                "cpu_baseline": cpu,
+                "small_m": small,
+            }
+            print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def time_e2e(torch, bw, p, steps, warmup, dist):
+    """Host buffers in, host buffers out, through the public API: per step a
+    pinned host->device copy of A, the GEMM, and a device->host copy of out."""
+    d = workloads.make(p)
+    A_host = torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).pin_memory()
+    out_host = torch.empty((p.M, p.N), dtype=torch.float16).pin_memory()
+    s = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+    packed = bw.pack(torch.from_numpy(d["codes"]).cuda(), p.mode)
+    A_dev = torch.empty((p.M, p.K), dtype=torch.float16, device="cuda")
+    out_dev = torch.empty((p.M, p.N), dtype=torch.float16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        A_dev.copy_(A_host, non_blocking=True)
+        bw.lowbit_gemm(A_dev, packed, s, p.mode, out=out_dev)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    secs = start.elapsed_time(end) / 1e3
+    t = torch.tensor([secs], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": flops(p) * steps * world / float(t.item()) / 1e12, "unit": UNIT,
+            "h2d_bytes_per_step": 2 * p.M * p.K, "d2h_bytes_per_step": 2 * p.M * p.N, "steps": steps}
+
+
+def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
+    """Bandwidth-bound regime: M=16.  64 rotating copies of the inputs
+    (about 500 MB, 4x L2) so that every launch reads its weights from HBM."""
+    sets = make_sets(p, 64, torch, bw, distinct_weights=False)
+    steps = max(args.steps, 200)
+    secs = time_launches(torch, bw, p, sets, steps, max(args.warmup, 10), dist)
+    t = torch.tensor([secs], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    per_launch = float(t.item()) / steps
+    nbytes = algorithmic_bytes(p)
+    achieved = nbytes / per_launch / 1e9
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    del sets
+    return {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "value": achieved, "unit": "GB/s",
+            "us_per_launch": per_launch * 1e6, "tflops": flops(p) / per_launch / 1e12,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}"),
+                         "algorithmic_bytes_per_launch": nbytes, "peak_source": f"{peaks_kind} hbm copy"},
+            "gpu_launches": steps}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_bonsai(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -205,7 +205,11 @@ def test_gemm_power_of_two_scaling_bitwise(mode):
     p = bw.pack(dev(d["codes"]), mode)
     one = bw.lowbit_gemm(A, p, s, mode)
     two = bw.lowbit_gemm(A * 2, p, s, mode)
-    assert torch.equal(two, one * 2)
+    # Doubling commutes with every FP32 partial sum and with the final FP16
+    # rounding, except where the result is FP16-subnormal (fixed 2^-24 grid).
+    normal = one.abs() >= 2.0 ** -14
+    assert normal.float().mean() > 0.99
+    assert torch.equal(two[normal], one[normal] * 2)
 
 
 @pytest.mark.parametrize("mode", ["binary", "ternary"])
@@ -222,7 +226,7 @@ def test_gemm_all_ones_closed_form(oracle_mod, mode):
     absw = (np.abs(c).reshape(N, K // 128, 128).sum(axis=2) * s.view(np.float16).astype(np.float64)).sum(axis=1)
     ref_bits = oracle_mod.double_to_half_bits(want)
     tol = RTOL * absw + oracle_mod.ulp16(ref_bits)
-    assert np.all(np.abs(got - want[None, :]) <= tol[None, :] + np.abs(want)[None, :] * 2.0 ** -11)
+    assert np.all(np.abs(got - want[None, :]) <= tol[None, :])
 
 
 def test_gemm_rows_independent():
