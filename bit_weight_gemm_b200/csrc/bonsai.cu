@@ -16,7 +16,6 @@ namespace bonsai {
 namespace {
 
 constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s: far above any launch's run time
-constexpr unsigned kErrBitTimeout = 1u << 7;             // set by wait_phase()
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -97,11 +96,74 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void*
 }
 
 // ------------------------------------------------------------------ GEMM --
-template <int MODE, int BLOCK_T, int STAGES>
+int sm_count() {
+  static int count[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (count[dev] == 0) {
+    int c = 0;
+    cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+    count[dev] = c > 0 ? c : 148;
+  }
+  return count[dev];
+}
+
+// Clusters of `ksplit` CTAs that can be resident at once (0 if unknown).
+template <int MODE, int BLOCK_T>
+int resident_clusters(int ksplit) {
+  using T = GemmTile<MODE, BLOCK_T>;
+  static std::mutex mu;
+  static int cache[9] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (ksplit < 1 || ksplit > 8) return 0;
+  if (cache[ksplit] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, ksplit);
+    cfg.blockDim = dim3(T::kThreads);
+    cfg.dynamicSmemBytes = T::kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 1;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = ksplit;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, lowbit_gemm_kernel<MODE, BLOCK_T>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = -1;
+    }
+    cache[ksplit] = n;
+  }
+  return cache[ksplit] > 0 ? cache[ksplit] : 0;
+}
+
+// Split K over a cluster when the tiles alone leave SMs idle: pick the split
+// that minimises waves x groups per CTA.
+template <int MODE, int BLOCK_T>
+int choose_ksplit(int tiles, int groups) {
+  const int sms = sm_count();
+  if (tiles >= sms) return 1;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int ks = 1; ks <= 8 && ks <= groups; ++ks) {
+    const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T>(ks);
+    if (per_wave <= 0) continue;
+    const int waves = (tiles + per_wave - 1) / per_wave;
+    const double cost = static_cast<double>(waves) * ((groups + ks - 1) / ks) + 0.25 * ks;  // small cost per split
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = ks;
+    }
+  }
+  return best;
+}
+
+template <int MODE, int BLOCK_T>
 int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, uint16_t* out,
                 cudaStream_t stream) {
-  using T = GemmTile<MODE, BLOCK_T, STAGES>;
-  auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T, STAGES>;
+  using T = GemmTile<MODE, BLOCK_T>;
+  auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -109,26 +171,61 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   });
   if (attr_err != cudaSuccess) return BONSAI_ERR_CUDA;
 
-  CUtensorMap map_act, map_w;
+  CUtensorMap map_act, map_w, map_out;
   const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
   if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, BLOCK_T, CU_TENSOR_MAP_SWIZZLE_128B))
     return BONSAI_ERR_CUDA;
   if (!make_map(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, words_per_row, N, T::kWordsPerGroup, T::kRows,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
+                MODE == BONSAI_BINARY ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_32B))
     return BONSAI_ERR_CUDA;
-  const dim3 grid((N + T::kRows - 1) / T::kRows, (M + BLOCK_T - 1) / BLOCK_T);
-  kernel<<<grid, 192, T::kSmemBytes, stream>>>(map_act, map_w, scales, out, M, N, K, kDefaultWaitLimitNs);
+  const bool tma_store = (N % 8) == 0;
+  if (tma_store) {
+    if (!make_map(&map_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, out, N, M, T::kRows, BLOCK_T,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return BONSAI_ERR_CUDA;
+  } else {
+    map_out = map_act;  // unused: rows of N halves are not 16-byte multiples, the kernel stores directly
+  }
+  const int groups = K / kGroup;
+  const int tiles_n = (N + T::kRows - 1) / T::kRows, tiles_m = (M + BLOCK_T - 1) / BLOCK_T;
+  const int ksplit = choose_ksplit<MODE, BLOCK_T>(tiles_n * tiles_m, groups);
+
+  GemmArgs args;
+  args.scales = scales;
+  args.out = out;
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.ksplit = ksplit;
+  args.tma_store = tma_store ? 1 : 0;
+  args.wait_limit_ns = kDefaultWaitLimitNs;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles_n, tiles_m, ksplit);
+  cfg.blockDim = dim3(T::kThreads);
+  cfg.dynamicSmemBytes = T::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  if (ksplit > 1) {
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 1;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = ksplit;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+  }
+  if (cudaLaunchKernelEx(&cfg, kernel, map_act, map_w, map_out, args) != cudaSuccess) return BONSAI_ERR_CUDA;
   return launch_status();
 }
 
 template <int MODE>
 int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
                   uint16_t* out, cudaStream_t stream) {
-  if (M <= 16) return launch_gemm<MODE, 16, 3>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 32) return launch_gemm<MODE, 32, 3>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 64) return launch_gemm<MODE, 64, 3>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 128) return launch_gemm<MODE, 128, 4>(A, packed, scales, M, N, K, out, stream);
-  return launch_gemm<MODE, 256, 3>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 16) return launch_gemm<MODE, 16>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 32) return launch_gemm<MODE, 32>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 64) return launch_gemm<MODE, 64>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 128) return launch_gemm<MODE, 128>(A, packed, scales, M, N, K, out, stream);
+  return launch_gemm<MODE, 256>(A, packed, scales, M, N, K, out, stream);
 }
 
 }  // namespace

@@ -2,28 +2,38 @@
 //
 // out[m,n] = sum_k A[m,k] * w[n,k],  w[n,k] = s[n,k/128] * t[n,k].
 //
-// Tile = 128 weight rows x BLOCK_T tokens, computed as D^T = W * A^T so that
-// the weights are the MMA's M side and can be fed from tensor memory:
+// A CTA computes a tile of 128 weight rows x BLOCK_T tokens over a range of
+// 128-wide K groups, as D^T = W * A^T, so that the weights are the MMA's M
+// side and can be fed from tensor memory.  Three rings decouple the stages:
 //
-//   warp 0      TMA producer: per 128-wide K group, the activation tile
-//               (BLOCK_T x 128 FP16, two 128-byte-swizzled K slices) and the
-//               packed words of the 128 weight rows land in a shared-memory
-//               stage; one mbarrier counts the bytes.
-//   warp 1      allocates tensor memory, then one thread issues
-//               tcgen05.mma.kind::f16 (M=128, N=BLOCK_T, K=16) x 8 per group:
-//               A = converted weights in TMEM, B = activations in SMEM,
-//               D = FP32 accumulator in TMEM; tcgen05.commit frees the stage.
-//   warps 2-5   converters: each thread owns one weight row (its TMEM lane),
-//               turns the group's packed words into exact FP16 products
-//               (binary: sign bit over s; ternary: the shifted 2-bit field is
-//               2t, times s) and stores them into the stage's TMEM columns
-//               with tcgen05.st.  After the last group they read the
-//               accumulator back (tcgen05.ld), scale by 1 (binary) or 1/2
-//               (ternary, exact), round once to FP16 and store out[m, n].
+//   act ring   (warp 0)  TMA of the activation tile per group: BLOCK_T rows
+//                        x 128 FP16 as two 128-byte-swizzled K slices.
+//   word ring  (warp 2)  TMA of the 128 rows' packed words per group
+//                        (32-byte swizzle for INT2 rows, so that the
+//                        converters' 16-byte reads are free of bank
+//                        conflicts).  Small, so it runs several groups ahead.
+//   TMEM ring  (warps 3-10, two per TMEM lane quadrant) converters: each
+//                        thread owns one weight row and half of a group's
+//                        words, turns them into exact FP16 products (binary:
+//                        sign bit over s; ternary: the shifted 2-bit field
+//                        is 2t, times s) and writes them to a TMEM stage
+//                        with tcgen05.st.
+//   warp 1               allocates TMEM; one thread issues
+//                        tcgen05.mma.kind::f16 (M=128, N=BLOCK_T, K=16) x 8
+//                        per group, A from TMEM, B from shared memory, FP32
+//                        accumulator in TMEM; tcgen05.commit releases the
+//                        act and TMEM stages.
+//
+// Epilogue, one CTA per tile (ksplit = 1): the converters read the
+// accumulator (tcgen05.ld), scale by 1 (binary) or 1/2 (ternary, exact),
+// round once to FP16 into a shared-memory tile, and one TMA store writes it.
+// Split K (ksplit > 1, small M): the ksplit CTAs of a cluster share a tile;
+// each leaves its FP32 partial in shared memory and, after a cluster
+// barrier, each reduces a slice of the tile from all partials over
+// distributed shared memory in a fixed order, rounds once and stores it.
 //
 // Weights are multiplied exactly: |t| <= 1 and s is FP16, so s*t (and 2*s*t
-// for |s| < 32768) is an FP16 value.  The sum runs in FP32 on the tensor
-// cores and is rounded to FP16 once.
+// for |s| < 32768) is an FP16 value; the sum runs in FP32.
 #pragma once
 
 #include "pack_dequant.cuh"
@@ -37,41 +47,45 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
   return p;
 }
 
-template <int MODE, int BLOCK_T, int STAGES>
+template <int MODE, int BLOCK_T>
 struct GemmTile {
-  static constexpr int kRows = 128;                                 // weight rows per tile (MMA M)
+  static constexpr int kRows = 128;  // weight rows per tile (MMA M)
   static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : 8;
-  static constexpr int kSliceBytes = BLOCK_T * 128;                 // BLOCK_T rows x 64 FP16
-  static constexpr int kActStageBytes = 2 * kSliceBytes;            // 128 K per stage
+  static constexpr int kSliceBytes = BLOCK_T * 128;       // BLOCK_T rows x 64 FP16
+  static constexpr int kActStageBytes = 2 * kSliceBytes;  // 128 K per stage
+  static constexpr int kActStages = BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : 6);
   static constexpr int kWStageBytes = kRows * kWordsPerGroup * 4;
-  static constexpr int kStageTx = kActStageBytes + kWStageBytes;
-  static constexpr int kACol0 = BLOCK_T < 64 ? 64 : BLOCK_T;        // TMEM columns: [0,BLOCK_T) = D
-  static constexpr int kTmemCols = pow2_at_least(kACol0 + STAGES * 64);
+  static constexpr int kWStages = (BLOCK_T >= 256 && MODE != BONSAI_BINARY) ? 6 : 8;
+  static constexpr int kTStages = 4;  // TMEM stages of converted weights, 64 columns each
+  static constexpr int kConvWarps = 8;
+  static constexpr int kThreads = 32 * (3 + kConvWarps);
+  static constexpr int kACol0 = BLOCK_T < 64 ? 64 : BLOCK_T;  // TMEM columns [0, BLOCK_T) hold D
+  static constexpr int kTmemCols = pow2_at_least(kACol0 + kTStages * 64);
   static constexpr int kActOff = 0;
-  static constexpr int kWOff = STAGES * kActStageBytes;
-  static constexpr int kBarOff = kWOff + STAGES * kWStageBytes;
-  static constexpr int kNumBars = 3 * STAGES + 1;
+  static constexpr int kWOff = kActStages * kActStageBytes;
+  static constexpr int kBarOff = kWOff + kWStages * kWStageBytes;
+  static constexpr int kNumBars = 2 * kActStages + 2 * kWStages + 2 * kTStages + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;          // + slack to align the base to 1024
-  // Shared memory also caps how many CTAs share an SM, so that their tensor
-  // memory allocations fit side by side (512 columns per SM, 228 KB of
-  // shared memory per SM): 512 columns -> 1 CTA, 256 -> 2.
-  static constexpr int kSmemFloor = kTmemCols == 512 ? 116 * 1024 : (kTmemCols == 256 ? 78 * 1024 : 0);
-  static constexpr int kSmemBytes = kSmemNeeded > kSmemFloor ? kSmemNeeded : kSmemFloor;
+  static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
+  // One CTA per SM: a second CTA could not get its 512 TMEM columns.
+  static constexpr int kSmemBytes = kSmemNeeded > 116 * 1024 ? kSmemNeeded : 116 * 1024;
+  static constexpr int kPartialStride = BLOCK_T + 1;  // floats per row of a split-K partial (padded)
   static constexpr float kOutScale = MODE == BONSAI_BINARY ? 1.0f : 0.5f;
   static_assert(BLOCK_T % 16 == 0 && BLOCK_T >= 16 && BLOCK_T <= 256, "MMA N for M=128");
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
-  static_assert(kTmemCols <= 512, "tensor memory has 512 columns");
+  static_assert(kTmemCols == 512, "one CTA per SM holds all of tensor memory");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+  static_assert(BLOCK_T * kRows * 2 <= kActStages * kActStageBytes, "output tile fits the act ring");
+  static_assert(kRows * kPartialStride * 4 <= kActStages * kActStageBytes, "partial fits the act ring");
 };
 
-// Converts one group (128 weights) of this thread's row into FP16 products
-// and writes them to 64 TMEM columns starting at `taddr`.
+// Converts half of a group of this thread's row (2 binary or 4 ternary
+// words) into FP16 products and writes them to 32 TMEM columns at `taddr`.
 template <int MODE>
-__device__ __forceinline__ void convert_group_to_tmem(const uint32_t* words, uint32_t s2, uint32_t taddr) {
+__device__ __forceinline__ void convert_half_group(const uint32_t* words, uint32_t s2, uint32_t taddr) {
   if (MODE == BONSAI_BINARY) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 2; ++j) {
       uint32_t v[16];
 #pragma unroll
       for (int p = 0; p < 16; ++p) v[p] = ((words[j] << p) & 0x80008000u) ^ s2;  // (+-s, +-s)
@@ -80,7 +94,7 @@ __device__ __forceinline__ void convert_group_to_tmem(const uint32_t* words, uin
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
       uint32_t v[8];
 #pragma unroll
       for (int p = 0; p < 8; ++p) v[p] = hmul2_bits((words[j] << (2 * p)) & 0xC000C000u, s2);  // (2ts, 2ts)
@@ -89,7 +103,7 @@ __device__ __forceinline__ void convert_group_to_tmem(const uint32_t* words, uin
   }
 }
 
-// Waits that the whole warp agrees on: every lane waits, and the warp goes on
+// A wait the whole warp agrees on: every lane waits, and the warp goes on
 // only if all lanes saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t limit_ns) {
@@ -97,19 +111,31 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int MODE, int BLOCK_T, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+struct GemmArgs {
+  const uint16_t* scales;
+  uint16_t* out;
+  int M, N, K;
+  int ksplit;     // CTAs along K sharing one tile (the cluster size along z)
+  int tma_store;  // 1: write the tile with one TMA store (needs N % 8 == 0)
+  uint64_t wait_limit_ns;
+};
+
+template <int MODE, int BLOCK_T>
+__global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_w,
-                       const uint16_t* __restrict__ scales, uint16_t* __restrict__ out, int M, int N, int K,
-                       uint64_t wait_limit_ns) {
-  using T = GemmTile<MODE, BLOCK_T, STAGES>;
+                       const __grid_constant__ CUtensorMap tmap_out, const GemmArgs args) {
+  using T = GemmTile<MODE, BLOCK_T>;
+  constexpr int AS = T::kActStages, WS = T::kWStages, TS = T::kTStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
-  const uint32_t full0 = smem_addr(bars);                 // full[s]:  TMA bytes of stage s landed
-  const uint32_t ready0 = smem_addr(bars + STAGES);       // ready[s]: converted weights in TMEM (4 warps)
-  const uint32_t empty0 = smem_addr(bars + 2 * STAGES);   // empty[s]: MMAs reading stage s finished
-  const uint32_t dfull = smem_addr(bars + 3 * STAGES);    // accumulator final
+  const uint32_t act_full0 = smem_addr(bars);                         // TMA bytes of act stage landed
+  const uint32_t act_empty0 = smem_addr(bars + AS);                   // MMAs reading act stage done
+  const uint32_t w_full0 = smem_addr(bars + 2 * AS);                  // TMA bytes of word stage landed
+  const uint32_t w_empty0 = smem_addr(bars + 2 * AS + WS);            // converters read word stage (8 warps)
+  const uint32_t t_ready0 = smem_addr(bars + 2 * AS + 2 * WS);        // converted weights in TMEM (8 warps)
+  const uint32_t t_free0 = smem_addr(bars + 2 * AS + 2 * WS + TS);    // MMAs reading TMEM stage done
+  const uint32_t dfull = smem_addr(bars + 2 * AS + 2 * WS + 2 * TS);  // accumulator final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::kMiscOff + 4);
 
@@ -117,13 +143,24 @@ __global__ void __launch_bounds__(192, 1)
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * T::kRows;
   const int m0 = blockIdx.y * BLOCK_T;
-  const int groups = K / kGroup;
+  const int groups = args.K / kGroup;
+  const int g_begin = static_cast<int>(static_cast<int64_t>(blockIdx.z) * groups / args.ksplit);
+  const int g_end = static_cast<int>(static_cast<int64_t>(blockIdx.z + 1) * groups / args.ksplit);
+  const int ng = g_end - g_begin;
+  const uint64_t limit = args.wait_limit_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(ready0 + 8 * s, 4);
-      mbar_init(empty0 + 8 * s, 1);
+    for (int s = 0; s < AS; ++s) {
+      mbar_init(act_full0 + 8 * s, 1);
+      mbar_init(act_empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < WS; ++s) {
+      mbar_init(w_full0 + 8 * s, 1);
+      mbar_init(w_empty0 + 8 * s, T::kConvWarps);
+    }
+    for (int s = 0; s < TS; ++s) {
+      mbar_init(t_ready0 + 8 * s, T::kConvWarps);
+      mbar_init(t_free0 + 8 * s, 1);
     }
     mbar_init(dfull, 1);
     *abort_flag = 0;
@@ -132,6 +169,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmap_act);
     tma_prefetch_map(&tmap_w);
+    tma_prefetch_map(&tmap_out);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), T::kTmemCols);
@@ -143,110 +181,189 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------------------------------------------------- producer
+    // ------------------------------------------------- activation producer
     if (elect_one()) {
       int issued = 0;
-      for (int g = 0; g < groups; ++g) {
-        const int s = g % STAGES;
-        const uint32_t ph = (g / STAGES) & 1;
-        if (!wait_phase(empty0 + 8 * s, ph ^ 1, abort_flag, wait_limit_ns)) break;
-        const uint32_t full = full0 + 8 * s;
-        mbar_arrive_expect_tx(full, T::kStageTx);
-        const uint32_t act = smem_addr(smem + T::kActOff + s * T::kActStageBytes);
-        tma_load_2d(act, &tmap_act, full, g * kGroup, m0);
-        tma_load_2d(act + T::kSliceBytes, &tmap_act, full, g * kGroup + 64, m0);
-        tma_load_2d(smem_addr(smem + T::kWOff + s * T::kWStageBytes), &tmap_w, full, g * T::kWordsPerGroup, n0);
-        issued = g + 1;
+      for (int i = 0; i < ng; ++i) {
+        const int s = i % AS;
+        if (!wait_phase(act_empty0 + 8 * s, ((i / AS) & 1) ^ 1, abort_flag, limit)) break;
+        const uint32_t full = act_full0 + 8 * s;
+        mbar_arrive_expect_tx(full, T::kActStageBytes);
+        const uint32_t dst = smem_addr(smem + T::kActOff + s * T::kActStageBytes);
+        const int k = (g_begin + i) * kGroup;
+        tma_load_2d(dst, &tmap_act, full, k, m0);
+        tma_load_2d(dst + T::kSliceBytes, &tmap_act, full, k + 64, m0);
+        issued = i + 1;
+      }
+      if (*abort_flag) {  // let copies in flight land before the CTA's memory goes away
+        for (int i = issued > AS ? issued - AS : 0; i < issued; ++i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(act_full0 + 8 * (i % AS), (i / AS) & 1) && global_timer_ns() - t0 < limit) {
+          }
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ packed-word producer
+    if (elect_one()) {
+      int issued = 0;
+      for (int i = 0; i < ng; ++i) {
+        const int s = i % WS;
+        if (!wait_phase(w_empty0 + 8 * s, ((i / WS) & 1) ^ 1, abort_flag, limit)) break;
+        const uint32_t full = w_full0 + 8 * s;
+        mbar_arrive_expect_tx(full, T::kWStageBytes);
+        tma_load_2d(smem_addr(smem + T::kWOff + s * T::kWStageBytes), &tmap_w, full,
+                    (g_begin + i) * T::kWordsPerGroup, n0);
+        issued = i + 1;
       }
       if (*abort_flag) {
-        // Let copies already in flight land before the CTA's memory goes away.
-        for (int g = issued - STAGES < 0 ? 0 : issued - STAGES; g < issued; ++g) {
+        for (int i = issued > WS ? issued - WS : 0; i < issued; ++i) {
           const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(full0 + 8 * (g % STAGES), (g / STAGES) & 1) && global_timer_ns() - t0 < wait_limit_ns) {
+          while (!mbar_try_wait(w_full0 + 8 * (i % WS), (i / WS) & 1) && global_timer_ns() - t0 < limit) {
           }
         }
       }
     }
   } else if (warp == 1) {
-    // --------------------------------------------------------- MMA issuer
+    // ---------------------------------------------------------- MMA issuer
     if (elect_one()) {
       constexpr uint32_t idesc = f16_instr_desc(128, BLOCK_T);
-      for (int g = 0; g < groups; ++g) {
-        const int s = g % STAGES;
-        const uint32_t ph = (g / STAGES) & 1;
-        if (!wait_phase(full0 + 8 * s, ph, abort_flag, wait_limit_ns)) break;
-        if (!wait_phase(ready0 + 8 * s, ph, abort_flag, wait_limit_ns)) break;
+      for (int i = 0; i < ng; ++i) {
+        const int sa = i % AS, st = i % TS;
+        if (!wait_phase(act_full0 + 8 * sa, (i / AS) & 1, abort_flag, limit)) break;
+        if (!wait_phase(t_ready0 + 8 * st, (i / TS) & 1, abort_flag, limit)) break;
         tc_fence_after_sync();
-        const uint32_t act = smem_addr(smem + T::kActOff + s * T::kActStageBytes);
-        const uint32_t a_cols = tmem + T::kACol0 + s * 64;
+        const uint32_t act = smem_addr(smem + T::kActOff + sa * T::kActStageBytes);
+        const uint32_t a_cols = tmem + T::kACol0 + st * 64;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sw128_kmajor_desc(act + (kk >> 2) * T::kSliceBytes + (kk & 3) * 32);
-          mma_f16_tmem_a(tmem, a_cols + kk * 8, bdesc, idesc, (g | kk) != 0 ? 1u : 0u);
+          mma_f16_tmem_a(tmem, a_cols + kk * 8, bdesc, idesc, (i | kk) != 0 ? 1u : 0u);
         }
-        mma_commit(empty0 + 8 * s);
+        mma_commit(act_empty0 + 8 * sa);
+        mma_commit(t_free0 + 8 * st);
       }
       mma_commit(dfull);  // also on abort: lets this thread see its MMAs drain
       if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(dfull, 0) && global_timer_ns() - t0 < wait_limit_ns) {
+        while (!mbar_try_wait(dfull, 0) && global_timer_ns() - t0 < limit) {
         }
       }
     }
   } else {
-    // ------------------------------------------------ converters + epilogue
+    // ------------------------------------------------ converters, epilogue
     const int quad = warp & 3;  // a warp may only touch TMEM lanes 32*(warp%4) .. +31
+    const int half = (warp - 3) >> 2;
     const int row = quad * 32 + lane;
     const int n = n0 + row;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint16_t* srow = scales + static_cast<size_t>(n) * groups;
-    uint32_t s_next = n < N ? __ldg(srow) : 0u;
+    const uint16_t* srow = args.scales + static_cast<size_t>(n) * groups + g_begin;
+    const bool row_ok = n < args.N;
+    uint32_t sq0 = row_ok ? __ldg(srow) : 0u;
+    uint32_t sq1 = (row_ok && ng > 1) ? __ldg(srow + 1) : 0u;
     bool ok = true;
-    for (int g = 0; g < groups; ++g) {
-      const int s = g % STAGES;
-      const uint32_t ph = (g / STAGES) & 1;
-      const uint32_t sc = s_next;
-      if (g + 1 < groups && n < N) s_next = __ldg(srow + g + 1);
-      ok = warp_wait(full0 + 8 * s, ph, abort_flag, wait_limit_ns) &&
-           warp_wait(empty0 + 8 * s, ph ^ 1, abort_flag, wait_limit_ns);
+    for (int i = 0; i < ng; ++i) {
+      const int sw = i % WS, st = i % TS;
+      const uint32_t sc = sq0;
+      sq0 = sq1;
+      sq1 = (row_ok && i + 2 < ng) ? __ldg(srow + i + 2) : 0u;
+      ok = warp_wait(w_full0 + 8 * sw, (i / WS) & 1, abort_flag, limit) &&
+           warp_wait(t_free0 + 8 * st, ((i / TS) & 1) ^ 1, abort_flag, limit);
       if (!ok) break;
-      tc_fence_after_sync();  // the MMAs that read this stage's columns are done
-      const uint4* src = reinterpret_cast<const uint4*>(smem + T::kWOff + s * T::kWStageBytes) +
-                         row * (T::kWordsPerGroup / 4);
-      uint32_t words[T::kWordsPerGroup];
-#pragma unroll
-      for (int i = 0; i < T::kWordsPerGroup / 4; ++i) {
-        const uint4 q = src[i];
-        words[4 * i] = q.x;
-        words[4 * i + 1] = q.y;
-        words[4 * i + 2] = q.z;
-        words[4 * i + 3] = q.w;
+      tc_fence_after_sync();  // the MMAs that read this TMEM stage are done
+      const uint8_t* wstage = smem + T::kWOff + sw * T::kWStageBytes;
+      uint32_t words[T::kWordsPerGroup / 2];
+      if (MODE == BONSAI_BINARY) {
+        const uint2 q = *reinterpret_cast<const uint2*>(wstage + row * 16 + half * 8);
+        words[0] = q.x;
+        words[1] = q.y;
+      } else {
+        // 32-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 2) & 1)
+        const int chunk = half ^ ((row >> 2) & 1);
+        const uint4 q = *reinterpret_cast<const uint4*>(wstage + row * 32 + chunk * 16);
+        words[0] = q.x;
+        words[1] = q.y;
+        words[2] = q.z;
+        words[3] = q.w;
       }
-      convert_group_to_tmem<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + s * 64);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(w_empty0 + 8 * sw);
+      convert_half_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64 + half * 32);
       tmem_store_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ready0 + 8 * s);
+      if (lane == 0) mbar_arrive(t_ready0 + 8 * st);
     }
-    if (ok && warp_wait(dfull, 0, abort_flag, wait_limit_ns)) {
-      tc_fence_after_sync();
+    if (ok) ok = warp_wait(dfull, 0, abort_flag, limit);
+    if (ok) tc_fence_after_sync();
+    constexpr int kHalfCols = BLOCK_T / 2;
+    const int c_begin = half * kHalfCols;
+    if (args.ksplit == 1) {
+      // FP16 tile [BLOCK_T tokens][128 rows] in the (now idle) act ring.
+      uint16_t* tile = reinterpret_cast<uint16_t*>(smem + T::kActOff);
+      if (ok) {
 #pragma unroll 1
-      for (int c = 0; c < BLOCK_T; c += 16) {
-        uint32_t v[16];
-        tmem_load_16(tmem + lane_base + c, v);
-        tmem_load_wait();
-        if (n < N) {
+        for (int c = 0; c < kHalfCols; c += 8) {
+          uint32_t v[8];
+          tmem_load_8(tmem + lane_base + c_begin + c, v);
+          tmem_load_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = m0 + c + j;
-            if (m < M) {
-              const __half h = __float2half_rn(__uint_as_float(v[j]) * T::kOutScale);
-              out[static_cast<size_t>(m) * N + n] = __half_as_ushort(h);
-            }
+          for (int j = 0; j < 8; ++j) {
+            const __half h = __float2half_rn(__uint_as_float(v[j]) * T::kOutScale);
+            tile[(c_begin + c + j) * T::kRows + row] = __half_as_ushort(h);
           }
         }
       }
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 32 * T::kConvWarps);
+      if (*abort_flag == 0) {
+        if (args.tma_store) {
+          if (warp == 3 && lane == 0) {
+            tma_store_2d(&tmap_out, smem_addr(tile), n0, m0);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+        } else {
+          const int ct = threadIdx.x - 96;  // 0 .. 255 over the converter warps
+          for (int e = ct; e < BLOCK_T * T::kRows; e += 32 * T::kConvWarps) {
+            const int m = m0 + e / T::kRows, nn = n0 + e % T::kRows;
+            if (m < args.M && nn < args.N) args.out[static_cast<size_t>(m) * args.N + nn] = tile[e];
+          }
+        }
+      }
+    } else if (ok) {
+      // FP32 partial [128 rows][BLOCK_T (+1 pad)] in the act ring.
+      float* part = reinterpret_cast<float*>(smem + T::kActOff);
+#pragma unroll 1
+      for (int c = 0; c < kHalfCols; c += 8) {
+        uint32_t v[8];
+        tmem_load_8(tmem + lane_base + c_begin + c, v);
+        tmem_load_wait();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part[row * T::kPartialStride + c_begin + c + j] = __uint_as_float(v[j]);
+      }
     }
+  }
+
+  if (args.ksplit > 1) {
+    __syncwarp();
+    cluster_sync();  // every partial of the cluster is written
+    if (*abort_flag == 0) {
+      const uint32_t part = smem_addr(smem + T::kActOff);
+      const int rank = static_cast<int>(cluster_ctarank());
+      constexpr int E = T::kRows * BLOCK_T;
+      const int e_begin = rank * E / args.ksplit, e_end = (rank + 1) * E / args.ksplit;
+      for (int e = e_begin + threadIdx.x; e < e_end; e += T::kThreads) {
+        const int m = e / T::kRows, r = e % T::kRows;  // consecutive threads: consecutive output columns
+        const uint32_t local = part + 4u * static_cast<uint32_t>(r * T::kPartialStride + m);
+        float sum = 0.0f;
+        for (int j = 0; j < args.ksplit; ++j) sum += ld_dsmem_f32(map_to_rank(local, j));
+        if (m0 + m < args.M && n0 + r < args.N)
+          args.out[static_cast<size_t>(m0 + m) * args.N + n0 + r] =
+              __half_as_ushort(__float2half_rn(sum * T::kOutScale));
+      }
+    }
+    cluster_sync();  // no CTA leaves while another still reads its partial
   }
 
   tc_fence_before_sync();

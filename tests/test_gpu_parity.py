@@ -122,6 +122,8 @@ SMALL_SHAPES = [
     (1, 8, 128), (5, 130, 256), (16, 128, 128), (17, 200, 384), (33, 256, 640), (64, 384, 256),
     (65, 129, 1152), (128, 256, 512), (129, 300, 256), (255, 128, 384), (256, 512, 256), (300, 384, 512),
     (513, 136, 768),
+    # few tiles, many groups: K is split over a cluster (sizes 2..8, not only powers of two)
+    (16, 256, 4096), (40, 384, 2048), (7, 128, 640), (100, 264, 1152), (16, 3072, 1024),
 ]
 
 
