@@ -344,7 +344,7 @@ def run_bonsai(args):
                 "warmup": args.warmup, "ms_per_step": result["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
                 "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "mode": p.mode, "group": 128,
-                           "parallelism": f"replicas{world}",
+                           "plan": bw.gemm_plan(p.M, p.N, p.K, p.mode), "parallelism": f"replicas{world}",
                            "l2": f"{args.sets} rotating input sets, {args.sets * (algorithmic_bytes(p)) / 1e6:.0f} MB "
                                  f"total > 126 MB L2"},
                 "roofline": {"bound": "tensor", "achieved": result["achieved"], "peak": result["peak"],
@@ -414,7 +414,8 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
     achieved = nbytes / per_launch / 1e9
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     del sets
-    return {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "value": achieved, "unit": "GB/s",
+    return {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "plan": bw.gemm_plan(p.M, p.N, p.K, p.mode),
+            "value": achieved, "unit": "GB/s",
             "us_per_launch": per_launch * 1e6, "tflops": flops(p) / per_launch / 1e12,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}"),

@@ -189,6 +189,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   const int groups = K / kGroup;
   const int tiles_n = (N + T::kRows - 1) / T::kRows, tiles_m = (M + BLOCK_T - 1) / BLOCK_T;
   const int ksplit = choose_ksplit<MODE, BLOCK_T>(tiles_n * tiles_m, groups);
+  if (ksplit > groups) return BONSAI_ERR_SHAPE;
 
   GemmArgs args;
   args.scales = scales;
@@ -216,6 +217,26 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   }
   if (cudaLaunchKernelEx(&cfg, kernel, map_act, map_w, map_out, args) != cudaSuccess) return BONSAI_ERR_CUDA;
   return launch_status();
+}
+
+struct Plan {
+  int block_t, ksplit, ctas;
+};
+
+template <int MODE, int BLOCK_T>
+Plan plan_for(int M, int N, int K) {
+  const int tiles = ((N + 127) / 128) * ((M + BLOCK_T - 1) / BLOCK_T);
+  const int ks = choose_ksplit<MODE, BLOCK_T>(tiles, K / kGroup);
+  return Plan{BLOCK_T, ks, tiles * ks};
+}
+
+template <int MODE>
+Plan plan_gemm(int M, int N, int K) {
+  if (M <= 16) return plan_for<MODE, 16>(M, N, K);
+  if (M <= 32) return plan_for<MODE, 32>(M, N, K);
+  if (M <= 64) return plan_for<MODE, 64>(M, N, K);
+  if (M <= 128) return plan_for<MODE, 128>(M, N, K);
+  return plan_for<MODE, 256>(M, N, K);
 }
 
 template <int MODE>
@@ -308,6 +329,26 @@ int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* sc
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   if (mode == BONSAI_BINARY) return dispatch_gemm<BONSAI_BINARY>(A, packed, scales, m, n, k, out, st);
   return dispatch_gemm<BONSAI_TERNARY_INT2>(A, packed, scales, m, n, k, out, st);
+}
+
+int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas) {
+  if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
+  int rc = check_shape(M, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (!block_t || !ksplit || !ctas) return BONSAI_ERR_INVALID_ARG;
+  if (M == 0 || N == 0 || K == 0) {
+    *block_t = 0;
+    *ksplit = 0;
+    *ctas = 0;
+    return BONSAI_OK;
+  }
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  const Plan p = mode == BONSAI_BINARY ? plan_gemm<BONSAI_BINARY>(m, n, k) : plan_gemm<BONSAI_TERNARY_INT2>(m, n, k);
+  *block_t = p.block_t;
+  *ksplit = p.ksplit;
+  *ctas = p.ctas;
+  return BONSAI_OK;
 }
 
 int bonsai_get_device_error(void) {

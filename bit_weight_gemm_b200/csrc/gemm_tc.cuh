@@ -55,7 +55,11 @@ struct GemmTile {
   static constexpr int kActStageBytes = 2 * kSliceBytes;  // 128 K per stage
   static constexpr int kActStages = BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : 6);
   static constexpr int kWStageBytes = kRows * kWordsPerGroup * 4;
-  static constexpr int kWStages = (BLOCK_T >= 256 && MODE != BONSAI_BINARY) ? 6 : 8;
+  // Small token tiles are bandwidth-bound: enough word stages to keep every
+  // load of a split-K CTA in flight at once.
+  static constexpr int kWStages = BLOCK_T <= 64 ? 16 : ((BLOCK_T >= 256 && MODE != BONSAI_BINARY) ? 6 : 8);
+  // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
+  static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
   static constexpr int kTStages = 4;  // TMEM stages of converted weights, 64 columns each
   static constexpr int kConvWarps = 8;
   static constexpr int kThreads = 32 * (3 + kConvWarps);
@@ -63,7 +67,8 @@ struct GemmTile {
   static constexpr int kTmemCols = pow2_at_least(kACol0 + kTStages * 64);
   static constexpr int kActOff = 0;
   static constexpr int kWOff = kActStages * kActStageBytes;
-  static constexpr int kBarOff = kWOff + kWStages * kWStageBytes;
+  static constexpr int kScaleOff = kWOff + kWStages * kWStageBytes;
+  static constexpr int kBarOff = kScaleOff + kScaleBytes;
   static constexpr int kNumBars = 2 * kActStages + 2 * kWStages + 2 * kTStages + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
@@ -259,14 +264,36 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint16_t* srow = args.scales + static_cast<size_t>(n) * groups + g_begin;
     const bool row_ok = n < args.N;
-    uint32_t sq0 = row_ok ? __ldg(srow) : 0u;
-    uint32_t sq1 = (row_ok && ng > 1) ? __ldg(srow + 1) : 0u;
+    // Scales: all of the tile's at once into shared memory when they fit
+    // (their loads overlap the first packed-word loads), else two groups
+    // ahead in registers.
+    const bool staged = T::kScaleBytes > 0 && T::kRows * ng * 2 <= T::kScaleBytes;
+    uint16_t* sstage = reinterpret_cast<uint16_t*>(smem + T::kScaleOff);
+    if (staged) {
+      const int ct = threadIdx.x - 96;  // 0 .. 255 over the converter warps
+      for (int e = ct; e < T::kRows * ng; e += 32 * T::kConvWarps) {
+        const int r = e / ng, g = e - (e / ng) * ng;
+        sstage[e] = (n0 + r < args.N) ? __ldg(args.scales + static_cast<size_t>(n0 + r) * groups + g_begin + g)
+                                      : uint16_t(0);
+      }
+      named_barrier_sync(2, 32 * T::kConvWarps);
+    }
+    uint32_t sq0 = 0, sq1 = 0;
+    if (!staged) {
+      sq0 = row_ok ? __ldg(srow) : 0u;
+      sq1 = (row_ok && ng > 1) ? __ldg(srow + 1) : 0u;
+    }
     bool ok = true;
     for (int i = 0; i < ng; ++i) {
       const int sw = i % WS, st = i % TS;
-      const uint32_t sc = sq0;
-      sq0 = sq1;
-      sq1 = (row_ok && i + 2 < ng) ? __ldg(srow + i + 2) : 0u;
+      uint32_t sc;
+      if (staged) {
+        sc = sstage[row * ng + i];
+      } else {
+        sc = sq0;
+        sq0 = sq1;
+        sq1 = (row_ok && i + 2 < ng) ? __ldg(srow + i + 2) : 0u;
+      }
       ok = warp_wait(w_full0 + 8 * sw, (i / WS) & 1, abort_flag, limit) &&
            warp_wait(t_free0 + 8 * st, ((i / TS) & 1) ^ 1, abort_flag, limit);
       if (!ok) break;
@@ -356,8 +383,13 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       for (int e = e_begin + threadIdx.x; e < e_end; e += T::kThreads) {
         const int m = e / T::kRows, r = e % T::kRows;  // consecutive threads: consecutive output columns
         const uint32_t local = part + 4u * static_cast<uint32_t>(r * T::kPartialStride + m);
-        float sum = 0.0f;
-        for (int j = 0; j < args.ksplit; ++j) sum += ld_dsmem_f32(map_to_rank(local, j));
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = j < args.ksplit ? ld_dsmem_f32(map_to_rank(local, j)) : 0.0f;
+        float sum = 0.0f;  // fixed order: CTA 0, 1, ...
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < args.ksplit) sum += v[j];
         if (m0 + m < args.M && n0 + r < args.N)
           args.out[static_cast<size_t>(m0 + m) * args.N + n0 + r] =
               __half_as_ushort(__float2half_rn(sum * T::kOutScale));

@@ -94,6 +94,13 @@ int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_
 int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int64_t M,
                        int64_t N, int64_t K, int mode, uint16_t* out, void* stream);
 
+/* The launch bonsai_lowbit_gemm makes for this problem on the current
+ * device: *block_t = tokens per tile (the MMA's N; each tile also covers 128
+ * weight rows), *ksplit = CTAs that share one tile along K as a thread-block
+ * cluster (1 = no split), *ctas = CTAs launched.  Host-side only (queries
+ * occupancy, launches nothing).  Zero-sized problems report zeros. */
+int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas);
+
 /* Reads and clears the device-side error word of the current device: 0 if
  * no kernel reported a problem since the last call, else a bonsai_status
  * (BONSAI_ERR_TIMEOUT when a bounded wait inside a kernel ran out; the

@@ -187,6 +187,15 @@ def test_gemm_full_size_sampled(oracle_mod, problem):
     assert np.isfinite(got.view(np.float16)).all()
 
 
+def test_plans_cover_both_epilogues():
+    big = bw.gemm_plan(4608, 9216, 3072, "ternary")
+    assert big == {"block_t": 256, "ksplit": 1, "ctas": 72 * 18}
+    for M, N, K in [(16, 3072, 9216), (16, 9216, 3072), (16, 256, 4096), (40, 384, 2048)]:
+        p = bw.gemm_plan(M, N, K, "ternary")
+        assert 1 < p["ksplit"] <= 8 and p["ctas"] % p["ksplit"] == 0, (M, N, K, p)
+    assert bw.gemm_plan(0, 8, 128, "binary") == {"block_t": 0, "ksplit": 0, "ctas": 0}
+
+
 # ------------------------------------------------------------ invariants
 @pytest.mark.parametrize("mode", ["binary", "ternary"])
 @pytest.mark.parametrize("M", [16, 200])
