@@ -63,7 +63,11 @@ struct GemmTile {
   static constexpr int kTStages = 4;  // TMEM stages of converted weights, 64 columns each
   static constexpr int kConvWarps = 8;
   static constexpr int kThreads = 32 * (3 + kConvWarps);
-  static constexpr int kACol0 = BLOCK_T < 64 ? 64 : BLOCK_T;  // TMEM columns [0, BLOCK_T) hold D
+  // Successive MMAs rotate over kAccs accumulators [a*BLOCK_T, (a+1)*BLOCK_T):
+  // with narrow tiles an MMA is a few cycles of work, so a chain of MMAs into
+  // one accumulator would run at the accumulate latency instead.
+  static constexpr int kAccs = BLOCK_T <= 32 ? 8 : 256 / BLOCK_T;
+  static constexpr int kACol0 = kAccs * BLOCK_T;  // converted-weight stages start after the accumulators
   static constexpr int kTmemCols = pow2_at_least(kACol0 + kTStages * 64);
   static constexpr int kActOff = 0;
   static constexpr int kWOff = kActStages * kActStageBytes;
@@ -114,6 +118,23 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
                                           uint64_t limit_ns) {
   const bool ok = wait_phase(bar, parity, abort_flag, limit_ns);
   return __all_sync(0xffffffffu, ok);
+}
+
+// Reads 8 columns of this thread's lane from each of the NACC accumulators
+// (NACC * BLOCK_T columns apart) and adds them in a fixed order.
+template <int NACC, int BLOCK_T>
+__device__ __forceinline__ void sum_accumulators(uint32_t taddr, float* acc) {
+  uint32_t v[NACC][8];
+#pragma unroll
+  for (int a = 0; a < NACC; ++a) tmem_load_8(taddr + a * BLOCK_T, v[a]);
+  tmem_load_wait();
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float x = __uint_as_float(v[0][j]);
+#pragma unroll
+    for (int a = 1; a < NACC; ++a) x += __uint_as_float(v[a][j]);
+    acc[j] = x;
+  }
 }
 
 struct GemmArgs {
@@ -243,7 +264,9 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sw128_kmajor_desc(act + (kk >> 2) * T::kSliceBytes + (kk & 3) * 32);
-          mma_f16_tmem_a(tmem, a_cols + kk * 8, bdesc, idesc, (i | kk) != 0 ? 1u : 0u);
+          const int step = i * 8 + kk;
+          const uint32_t d = tmem + (step % T::kAccs) * BLOCK_T;
+          mma_f16_tmem_a(d, a_cols + kk * 8, bdesc, idesc, step >= T::kAccs ? 1u : 0u);
         }
         mma_commit(act_empty0 + 8 * sa);
         mma_commit(t_free0 + 8 * st);
@@ -331,12 +354,11 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       if (ok) {
 #pragma unroll 1
         for (int c = 0; c < kHalfCols; c += 8) {
-          uint32_t v[8];
-          tmem_load_8(tmem + lane_base + c_begin + c, v);
-          tmem_load_wait();
+          float acc[8];
+          sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, acc);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const __half h = __float2half_rn(__uint_as_float(v[j]) * T::kOutScale);
+            const __half h = __float2half_rn(acc[j] * T::kOutScale);
             tile[(c_begin + c + j) * T::kRows + row] = __half_as_ushort(h);
           }
         }
@@ -363,11 +385,10 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       float* part = reinterpret_cast<float*>(smem + T::kActOff);
 #pragma unroll 1
       for (int c = 0; c < kHalfCols; c += 8) {
-        uint32_t v[8];
-        tmem_load_8(tmem + lane_base + c_begin + c, v);
-        tmem_load_wait();
+        float acc[8];
+        sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, acc);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) part[row * T::kPartialStride + c_begin + c + j] = __uint_as_float(v[j]);
+        for (int j = 0; j < 8; ++j) part[row * T::kPartialStride + c_begin + c + j] = acc[j];
       }
     }
   }
