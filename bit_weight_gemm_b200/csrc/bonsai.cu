@@ -81,18 +81,79 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps are kept in a small cache: encoding costs
+// microseconds of host time per call, comparable to a small-M launch.  A map
+// holds only an address, sizes and a box shape, so a hit is always valid.
+struct MapKey {
+  const void* base;
+  uint64_t inner, rows;
+  uint32_t box_inner, box_rows;
+  int dtype, swizzle, device;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && inner == o.inner && rows == o.rows && box_inner == o.box_inner &&
+           box_rows == o.box_rows && dtype == o.dtype && swizzle == o.swizzle && device == o.device;
+  }
+};
+
+constexpr int kMapCacheSize = 256;
+struct MapCache {
+  std::mutex mu;
+  MapKey keys[kMapCacheSize];
+  CUtensorMap maps[kMapCacheSize];
+  bool used[kMapCacheSize] = {};
+  int next = 0;
+};
+
+MapCache& map_cache() {
+  static MapCache cache;
+  return cache;
+}
+
 // Row-major 2-D tensor [rows, inner] of `elem` bytes per element, copied in
 // boxes of box_rows x box_inner.
 bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void* base, uint64_t inner,
               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  int device = 0;
+  cudaGetDevice(&device);
+  const MapKey key{base, inner, rows, box_inner, box_rows, static_cast<int>(dtype), static_cast<int>(swizzle), device};
+  MapCache& cache = map_cache();
+  uint64_t h = reinterpret_cast<uintptr_t>(base) * 0x9E3779B97F4A7C15ull;
+  h ^= (inner * 0xC2B2AE3D27D4EB4Full) ^ (rows * 0x165667B19E3779F9ull) ^
+       (static_cast<uint64_t>(box_inner) << 40) ^ (static_cast<uint64_t>(box_rows) << 20) ^
+       (static_cast<uint64_t>(dtype) << 8) ^ static_cast<uint64_t>(swizzle) ^ (static_cast<uint64_t>(device) << 56);
+  const int home = static_cast<int>((h >> 32) % kMapCacheSize);
+  constexpr int kProbe = 8;
+  {
+    std::lock_guard<std::mutex> lock(cache.mu);
+    for (int i = 0; i < kProbe; ++i) {
+      const int slot = (home + i) % kMapCacheSize;
+      if (cache.used[slot] && cache.keys[slot] == key) {
+        *map = cache.maps[slot];
+        return true;
+      }
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem)};
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(cache.mu);
+  int slot = -1;
+  for (int i = 0; i < kProbe && slot < 0; ++i)
+    if (!cache.used[(home + i) % kMapCacheSize]) slot = (home + i) % kMapCacheSize;
+  if (slot < 0) {  // all probe slots taken: replace them in turn
+    slot = (home + cache.next) % kMapCacheSize;
+    cache.next = (cache.next + 1) % kProbe;
+  }
+  cache.keys[slot] = key;
+  cache.maps[slot] = *map;
+  cache.used[slot] = true;
+  return true;
 }
 
 // ------------------------------------------------------------------ GEMM --
