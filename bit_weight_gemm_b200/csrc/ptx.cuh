@@ -72,12 +72,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Waits until the phase with the given parity of barrier `bar` completes.
-// Returns false (without waiting further) when the CTA's abort flag is up or
-// when `limit_ns` has passed; in the latter case it records the timeout.
-__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                        uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Non-blocking test: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "  selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// The blocking part of wait_phase, kept out of line.
+__device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -90,6 +102,16 @@ __device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile 
       }
     }
   }
+}
+
+// Waits until the phase with the given parity of barrier `bar` completes.
+// Returns false (without waiting further) when the CTA's abort flag is up or
+// when `limit_ns` has passed; in the latter case it records the timeout.
+// A phase that has already completed costs one non-blocking test.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return wait_phase_slow(bar, parity, abort_flag, limit_ns);
 }
 
 // ------------------------------------------------------------------ TMA --
