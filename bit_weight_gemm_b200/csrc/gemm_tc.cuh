@@ -12,12 +12,14 @@
 //                        (32-byte swizzle for INT2 rows, so that the
 //                        converters' 16-byte reads are free of bank
 //                        conflicts).  Small, so it runs several groups ahead.
-//   TMEM ring  (warps 3-10, two per TMEM lane quadrant) converters: each
-//                        thread owns one weight row and half of a group's
-//                        words, turns them into exact FP16 products (binary:
-//                        sign bit over s; ternary: the shifted 2-bit field
-//                        is 2t, times s) and writes them to a TMEM stage
-//                        with tcgen05.st.
+//   TMEM ring  (warps 3-10, two per TMEM lane quadrant, taking alternate
+//                        groups) converters: each thread owns one weight row,
+//                        turns the group's words into exact FP16 products
+//                        (binary: sign bit over s; ternary: the shifted 2-bit
+//                        field is 2t, times s) and writes them to a TMEM
+//                        stage with tcgen05.st.  Stage s of the act ring and
+//                        of the TMEM ring hold the same group and are
+//                        released by one tcgen05.commit.
 //   warp 1               allocates TMEM; one thread issues
 //                        tcgen05.mma.kind::f16 (M=128, N=BLOCK_T, K=16) x 8
 //                        per group, A from TMEM, B from shared memory, FP32
@@ -30,7 +32,9 @@
 // Split K (ksplit > 1, small M): the ksplit CTAs of a cluster share a tile;
 // each leaves its FP32 partial in shared memory and, after a cluster
 // barrier, each reduces a slice of the tile from all partials over
-// distributed shared memory in a fixed order, rounds once and stores it.
+// distributed shared memory (16-byte loads) in a fixed order, rounds once
+// and stores it.  Accumulation is spread over several TMEM accumulators so
+// that narrow MMAs do not queue behind one accumulator.
 //
 // Weights are multiplied exactly: |t| <= 1 and s is FP16, so s*t (and 2*s*t
 // for |s| < 32768) is an FP16 value; the sum runs in FP32.
@@ -81,23 +85,23 @@ struct GemmTile {
   static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
   // One CTA per SM: a second CTA could not get its 512 TMEM columns.
   static constexpr int kSmemBytes = kSmemNeeded > 116 * 1024 ? kSmemNeeded : 116 * 1024;
-  static constexpr int kPartialStride = BLOCK_T + 1;  // floats per row of a split-K partial (padded)
+
   static constexpr float kOutScale = MODE == BONSAI_BINARY ? 1.0f : 0.5f;
   static_assert(BLOCK_T % 16 == 0 && BLOCK_T >= 16 && BLOCK_T <= 256, "MMA N for M=128");
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kTmemCols == 512, "one CTA per SM holds all of tensor memory");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(BLOCK_T * kRows * 2 <= kActStages * kActStageBytes, "output tile fits the act ring");
-  static_assert(kRows * kPartialStride * 4 <= kActStages * kActStageBytes, "partial fits the act ring");
+  static_assert(kRows * BLOCK_T * 4 <= kActStages * kActStageBytes, "partial fits the act ring");
 };
 
-// Converts half of a group of this thread's row (2 binary or 4 ternary
-// words) into FP16 products and writes them to 32 TMEM columns at `taddr`.
+// Converts one group of this thread's row (4 binary or 8 ternary words)
+// into FP16 products and writes them to 64 TMEM columns at `taddr`.
 template <int MODE>
-__device__ __forceinline__ void convert_half_group(const uint32_t* words, uint32_t s2, uint32_t taddr) {
+__device__ __forceinline__ void convert_group(const uint32_t* words, uint32_t s2, uint32_t taddr) {
   if (MODE == BONSAI_BINARY) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < 4; ++j) {
       uint32_t v[16];
 #pragma unroll
       for (int p = 0; p < 16; ++p) v[p] = ((words[j] << p) & 0x80008000u) ^ s2;  // (+-s, +-s)
@@ -106,7 +110,7 @@ __device__ __forceinline__ void convert_half_group(const uint32_t* words, uint32
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 8; ++j) {
       uint32_t v[8];
 #pragma unroll
       for (int p = 0; p < 8; ++p) v[p] = hmul2_bits((words[j] << (2 * p)) & 0xC000C000u, s2);  // (2ts, 2ts)
@@ -180,12 +184,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(act_full0 + 8 * s, 1);
-      mbar_init(t_ready0 + 8 * s, T::kConvWarps);
+      mbar_init(t_ready0 + 8 * s, 4);  // one converter warp per TMEM lane quadrant
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int s = 0; s < WS; ++s) {
       mbar_init(w_full0 + 8 * s, 1);
-      mbar_init(w_empty0 + 8 * s, T::kConvWarps);
+      mbar_init(w_empty0 + 8 * s, 4);
     }
     mbar_init(dfull, 1);
     *abort_flag = 0;
@@ -283,6 +287,8 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------ converters, epilogue
+    // The two warps of a TMEM lane quadrant take alternate groups, so that
+    // one's barrier waits overlap the other's conversion.
     const int quad = warp & 3;  // a warp may only touch TMEM lanes 32*(warp%4) .. +31
     const int half = (warp - 3) >> 2;
     const int row = quad * 32 + lane;
@@ -305,12 +311,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       named_barrier_sync(2, 32 * T::kConvWarps);
     }
     uint32_t sq0 = 0, sq1 = 0;
-    if (!staged) {
-      sq0 = row_ok ? __ldg(srow) : 0u;
-      sq1 = (row_ok && ng > 1) ? __ldg(srow + 1) : 0u;
-    }
     bool ok = true;
-    for (int i = 0; i < ng; ++i) {
+    if (!staged) {
+      sq0 = (row_ok && half < ng) ? __ldg(srow + half) : 0u;
+      sq1 = (row_ok && half + 2 < ng) ? __ldg(srow + half + 2) : 0u;
+    }
+    for (int i = half; i < ng; i += 2) {
       const int sw = i % WS, st = i % S;
       uint32_t sc;
       if (staged) {
@@ -318,30 +324,37 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       } else {
         sc = sq0;
         sq0 = sq1;
-        sq1 = (row_ok && i + 2 < ng) ? __ldg(srow + i + 2) : 0u;
+        sq1 = (row_ok && i + 4 < ng) ? __ldg(srow + i + 4) : 0u;
       }
       ok = warp_wait(w_full0 + 8 * sw, (i / WS) & 1, abort_flag, limit) &&
            warp_wait(empty0 + 8 * st, ((i / S) & 1) ^ 1, abort_flag, limit);
       if (!ok) break;
       tc_fence_after_sync();  // the MMAs that read this TMEM stage are done
       const uint8_t* wstage = smem + T::kWOff + sw * T::kWStageBytes;
-      uint32_t words[T::kWordsPerGroup / 2];
+      uint32_t words[T::kWordsPerGroup];
       if (MODE == BONSAI_BINARY) {
-        const uint2 q = *reinterpret_cast<const uint2*>(wstage + row * 16 + half * 8);
-        words[0] = q.x;
-        words[1] = q.y;
-      } else {
-        // 32-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 2) & 1)
-        const int chunk = half ^ ((row >> 2) & 1);
-        const uint4 q = *reinterpret_cast<const uint4*>(wstage + row * 32 + chunk * 16);
+        const uint4 q = *reinterpret_cast<const uint4*>(wstage + row * 16);
         words[0] = q.x;
         words[1] = q.y;
         words[2] = q.z;
         words[3] = q.w;
+      } else {
+        // 32-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 2) & 1)
+        const int flip = (row >> 2) & 1;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(wstage + row * 32 + flip * 16);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(wstage + row * 32 + (flip ^ 1) * 16);
+        words[0] = q0.x;
+        words[1] = q0.y;
+        words[2] = q0.z;
+        words[3] = q0.w;
+        words[4] = q1.x;
+        words[5] = q1.y;
+        words[6] = q1.z;
+        words[7] = q1.w;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(w_empty0 + 8 * sw);
-      convert_half_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64 + half * 32);
+      convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
       tmem_store_wait();
       tc_fence_before_sync();
       __syncwarp();
@@ -384,14 +397,14 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
         }
       }
     } else if (ok) {
-      // FP32 partial [128 rows][BLOCK_T (+1 pad)] in the act ring.
+      // FP32 partial [BLOCK_T tokens][128 rows] in the act ring.
       float* part = reinterpret_cast<float*>(smem + T::kActOff);
 #pragma unroll 1
       for (int c = 0; c < kHalfCols; c += 8) {
         float acc[8];
         sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, acc);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) part[row * T::kPartialStride + c_begin + c + j] = acc[j];
+        for (int j = 0; j < 8; ++j) part[(c_begin + c + j) * T::kRows + row] = acc[j];
       }
     }
   }
@@ -400,23 +413,36 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     __syncwarp();
     cluster_sync();  // every partial of the cluster is written
     if (*abort_flag == 0) {
+      // This CTA's share of the tile, in runs of 4 consecutive rows of one
+      // token: 16-byte loads from every CTA's partial, added in rank order.
       const uint32_t part = smem_addr(smem + T::kActOff);
       const int rank = static_cast<int>(cluster_ctarank());
-      constexpr int E = T::kRows * BLOCK_T;
-      const int e_begin = rank * E / args.ksplit, e_end = (rank + 1) * E / args.ksplit;
-      for (int e = e_begin + threadIdx.x; e < e_end; e += T::kThreads) {
-        const int m = e / T::kRows, r = e % T::kRows;  // consecutive threads: consecutive output columns
-        const uint32_t local = part + 4u * static_cast<uint32_t>(r * T::kPartialStride + m);
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = j < args.ksplit ? ld_dsmem_f32(map_to_rank(local, j)) : 0.0f;
-        float sum = 0.0f;  // fixed order: CTA 0, 1, ...
+      constexpr int Q = T::kRows * BLOCK_T / 4;
+      const int q_begin = rank * Q / args.ksplit, q_end = (rank + 1) * Q / args.ksplit;
+      for (int q = q_begin + threadIdx.x; q < q_end; q += T::kThreads) {
+        const int m = (4 * q) / T::kRows, r = (4 * q) % T::kRows;
+        const uint32_t local = part + 16u * static_cast<uint32_t>(q);
+        float4 v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (j < args.ksplit) sum += v[j];
-        if (m0 + m < args.M && n0 + r < args.N)
-          args.out[static_cast<size_t>(m0 + m) * args.N + n0 + r] =
-              __half_as_ushort(__float2half_rn(sum * T::kOutScale));
+          if (j < args.ksplit) v[j] = ld_dsmem_f32x4(map_to_rank(local, j));
+        float4 sum = v[0];
+#pragma unroll
+        for (int j = 1; j < 8; ++j)
+          if (j < args.ksplit) {
+            sum.x += v[j].x;
+            sum.y += v[j].y;
+            sum.z += v[j].z;
+            sum.w += v[j].w;
+          }
+        const int gm = m0 + m;
+        if (gm < args.M) {
+          const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+          uint16_t* dst = args.out + static_cast<size_t>(gm) * args.N + n0 + r;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (n0 + r + j < args.N) dst[j] = __half_as_ushort(__float2half_rn(vals[j] * T::kOutScale));
+        }
       }
     }
     cluster_sync();  // no CTA leaves while another still reads its partial
