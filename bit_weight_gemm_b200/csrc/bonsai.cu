@@ -236,8 +236,8 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
   if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, BLOCK_T, CU_TENSOR_MAP_SWIZZLE_128B))
     return BONSAI_ERR_CUDA;
-  if (!make_map(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, words_per_row, N, T::kWordsPerGroup, T::kRows,
-                MODE == BONSAI_BINARY ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_32B))
+  if (!make_map(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, words_per_row, N, 32, T::kRows,
+                CU_TENSOR_MAP_SWIZZLE_128B))
     return BONSAI_ERR_CUDA;
   const bool tma_store = (N % 8) == 0;
   if (tma_store) {

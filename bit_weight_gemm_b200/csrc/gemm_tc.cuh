@@ -8,10 +8,11 @@
 //
 //   act ring   (warp 0)  TMA of the activation tile per group: BLOCK_T rows
 //                        x 128 FP16 as two 128-byte-swizzled K slices.
-//   word ring  (warp 2)  TMA of the 128 rows' packed words per group
-//                        (32-byte swizzle for INT2 rows, so that the
-//                        converters' 16-byte reads are free of bank
-//                        conflicts).  Small, so it runs several groups ahead.
+//   word ring  (warp 2)  TMA of the 128 rows' packed words, 128 bytes of
+//                        each row per stage (4 ternary or 8 binary groups)
+//                        with 128-byte swizzling, so that the converters'
+//                        16-byte reads are free of bank conflicts and each
+//                        request moves a whole 128-byte line.
 //   TMEM ring  (warps 3-10, two per TMEM lane quadrant, taking alternate
 //                        groups) converters: each thread owns one weight row,
 //                        turns the group's words into exact FP16 products
@@ -61,10 +62,13 @@ struct GemmTile {
   // and are released together by one tcgen05.commit.
   static constexpr int kStages = BLOCK_T >= 256 ? 3 : 4;
   static constexpr int kActStages = kStages;
-  static constexpr int kWStageBytes = kRows * kWordsPerGroup * 4;
+  // A word stage is 128 bytes of every row: 4 ternary or 8 binary groups,
+  // one TMA box with 128-byte swizzling.
+  static constexpr int kWGroups = 32 / kWordsPerGroup;
+  static constexpr int kWStageBytes = kRows * 128;
   // Small token tiles are bandwidth-bound: enough word stages to keep every
   // load of a split-K CTA in flight at once.
-  static constexpr int kWStages = BLOCK_T <= 64 ? 16 : ((BLOCK_T >= 256 && MODE != BONSAI_BINARY) ? 6 : 8);
+  static constexpr int kWStages = BLOCK_T >= 256 ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
   static constexpr int kTStages = kStages;  // TMEM stages of converted weights, 64 columns each
@@ -189,7 +193,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     }
     for (int s = 0; s < WS; ++s) {
       mbar_init(w_full0 + 8 * s, 1);
-      mbar_init(w_empty0 + 8 * s, 4);
+      mbar_init(w_empty0 + 8 * s, T::kConvWarps);  // every converter warp reads each full stage
     }
     mbar_init(dfull, 1);
     *abort_flag = 0;
@@ -236,13 +240,14 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     // ------------------------------------------------ packed-word producer
     if (elect_one()) {
       int issued = 0;
-      for (int i = 0; i < ng; ++i) {
+      const int nw = (ng + T::kWGroups - 1) / T::kWGroups;
+      for (int i = 0; i < nw; ++i) {
         const int s = i % WS;
         if (!wait_phase(w_empty0 + 8 * s, ((i / WS) & 1) ^ 1, abort_flag, limit)) break;
         const uint32_t full = w_full0 + 8 * s;
         mbar_arrive_expect_tx(full, T::kWStageBytes);
         tma_load_2d(smem_addr(smem + T::kWOff + s * T::kWStageBytes), &tmap_w, full,
-                    (g_begin + i) * T::kWordsPerGroup, n0);
+                    (g_begin + i * T::kWGroups) * T::kWordsPerGroup, n0);
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -317,7 +322,8 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       sq1 = (row_ok && half + 2 < ng) ? __ldg(srow + half + 2) : 0u;
     }
     for (int i = half; i < ng; i += 2) {
-      const int sw = i % WS, st = i % S;
+      const int wj = i / T::kWGroups;  // word stage of this group
+      const int sw = wj % WS, st = i % S;
       uint32_t sc;
       if (staged) {
         sc = sstage[row * ng + i];
@@ -326,23 +332,24 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
         sq0 = sq1;
         sq1 = (row_ok && i + 4 < ng) ? __ldg(srow + i + 4) : 0u;
       }
-      ok = warp_wait(w_full0 + 8 * sw, (i / WS) & 1, abort_flag, limit) &&
+      ok = warp_wait(w_full0 + 8 * sw, (wj / WS) & 1, abort_flag, limit) &&
            warp_wait(empty0 + 8 * st, ((i / S) & 1) ^ 1, abort_flag, limit);
       if (!ok) break;
       tc_fence_after_sync();  // the MMAs that read this TMEM stage are done
       const uint8_t* wstage = smem + T::kWOff + sw * T::kWStageBytes;
+      // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
+      const int pos = i % T::kWGroups;
+      const uint8_t* wrow = wstage + row * 128;
       uint32_t words[T::kWordsPerGroup];
       if (MODE == BONSAI_BINARY) {
-        const uint4 q = *reinterpret_cast<const uint4*>(wstage + row * 16);
+        const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16 * (pos ^ (row & 7)));
         words[0] = q.x;
         words[1] = q.y;
         words[2] = q.z;
         words[3] = q.w;
       } else {
-        // 32-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 2) & 1)
-        const int flip = (row >> 2) & 1;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(wstage + row * 32 + flip * 16);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(wstage + row * 32 + (flip ^ 1) * 16);
+        const uint4 q0 = *reinterpret_cast<const uint4*>(wrow + 16 * ((2 * pos) ^ (row & 7)));
+        const uint4 q1 = *reinterpret_cast<const uint4*>(wrow + 16 * ((2 * pos + 1) ^ (row & 7)));
         words[0] = q0.x;
         words[1] = q0.y;
         words[2] = q0.z;
@@ -353,7 +360,9 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
         words[7] = q1.w;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(w_empty0 + 8 * sw);
+      // Release the word stage after this warp's last group in it.
+      const int stage_end = (wj + 1) * T::kWGroups < ng ? (wj + 1) * T::kWGroups : ng;
+      if (lane == 0 && i + 2 >= stage_end) mbar_arrive(w_empty0 + 8 * sw);
       convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
       tmem_store_wait();
       tc_fence_before_sync();
