@@ -18,9 +18,7 @@
 //                        turns the group's words into exact FP16 products
 //                        (binary: sign bit over s; ternary: the shifted 2-bit
 //                        field is 2t, times s) and writes them to a TMEM
-//                        stage with tcgen05.st.  Stage s of the act ring and
-//                        of the TMEM ring hold the same group and are
-//                        released by one tcgen05.commit.
+//                        stage with tcgen05.st.
 //   warp 1               allocates TMEM; one thread issues
 //                        tcgen05.mma.kind::f16 (M=128, N=BLOCK_T, K=16) x 8
 //                        per group, A from TMEM, B from shared memory, FP32
@@ -58,10 +56,9 @@ struct GemmTile {
   static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : 8;
   static constexpr int kSliceBytes = BLOCK_T * 128;       // BLOCK_T rows x 64 FP16
   static constexpr int kActStageBytes = 2 * kSliceBytes;  // 128 K per stage
-  // Stage s of the act ring and stage s of the TMEM ring feed the same group
-  // and are released together by one tcgen05.commit.
-  static constexpr int kStages = BLOCK_T >= 256 ? 3 : 4;
-  static constexpr int kActStages = kStages;
+  // Activation stages: as many as fit next to the word ring and the scales,
+  // so that narrow tiles keep a split-K CTA's whole K range in flight.
+  static constexpr int kActStages = BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : (96 * 1024) / kActStageBytes);
   // A word stage is 128 bytes of every row: 4 ternary or 8 binary groups,
   // one TMA box with 128-byte swizzling.
   static constexpr int kWGroups = 32 / kWordsPerGroup;
@@ -71,7 +68,7 @@ struct GemmTile {
   static constexpr int kWStages = BLOCK_T >= 256 ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
-  static constexpr int kTStages = kStages;  // TMEM stages of converted weights, 64 columns each
+  static constexpr int kTStages = BLOCK_T >= 256 ? 3 : 4;  // TMEM stages of converted weights, 64 columns each
   static constexpr int kConvWarps = 8;
   static constexpr int kThreads = 32 * (3 + kConvWarps);
   // Successive MMAs rotate over kAccs accumulators [a*BLOCK_T, (a+1)*BLOCK_T):
@@ -84,7 +81,7 @@ struct GemmTile {
   static constexpr int kWOff = kActStages * kActStageBytes;
   static constexpr int kScaleOff = kWOff + kWStages * kWStageBytes;
   static constexpr int kBarOff = kScaleOff + kScaleBytes;
-  static constexpr int kNumBars = 3 * kStages + 2 * kWStages + 1;
+  static constexpr int kNumBars = 2 * kActStages + 2 * kTStages + 2 * kWStages + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
   // One CTA per SM: a second CTA could not get its 512 TMEM columns.
@@ -162,16 +159,17 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_out, const GemmArgs args) {
   using T = GemmTile<MODE, BLOCK_T>;
-  constexpr int S = T::kStages, WS = T::kWStages;
+  constexpr int AS = T::kActStages, TS = T::kTStages, WS = T::kWStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
-  const uint32_t act_full0 = smem_addr(bars);                 // TMA bytes of act stage s landed
-  const uint32_t t_ready0 = smem_addr(bars + S);              // converted weights in TMEM stage s (8 warps)
-  const uint32_t empty0 = smem_addr(bars + 2 * S);            // MMAs reading act + TMEM stage s done
-  const uint32_t w_full0 = smem_addr(bars + 3 * S);           // TMA bytes of word stage landed
-  const uint32_t w_empty0 = smem_addr(bars + 3 * S + WS);     // converters read word stage (8 warps)
-  const uint32_t dfull = smem_addr(bars + 3 * S + 2 * WS);    // accumulator final
+  const uint32_t act_full0 = smem_addr(bars);                     // TMA bytes of act stage landed
+  const uint32_t act_empty0 = smem_addr(bars + AS);               // MMAs reading act stage done
+  const uint32_t t_ready0 = smem_addr(bars + 2 * AS);             // converted weights in TMEM stage (4 warps)
+  const uint32_t t_free0 = smem_addr(bars + 2 * AS + TS);         // MMAs reading TMEM stage done
+  const uint32_t w_full0 = smem_addr(bars + 2 * AS + 2 * TS);     // TMA bytes of word stage landed
+  const uint32_t w_empty0 = smem_addr(bars + 2 * AS + 2 * TS + WS);  // converters read word stage
+  const uint32_t dfull = smem_addr(bars + 2 * AS + 2 * TS + 2 * WS);  // accumulator final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::kMiscOff + 4);
 
@@ -186,10 +184,13 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
   const uint64_t limit = args.wait_limit_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < AS; ++s) {
       mbar_init(act_full0 + 8 * s, 1);
+      mbar_init(act_empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < TS; ++s) {
       mbar_init(t_ready0 + 8 * s, 4);  // one converter warp per TMEM lane quadrant
-      mbar_init(empty0 + 8 * s, 1);
+      mbar_init(t_free0 + 8 * s, 1);
     }
     for (int s = 0; s < WS; ++s) {
       mbar_init(w_full0 + 8 * s, 1);
@@ -218,8 +219,8 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     if (elect_one()) {
       int issued = 0;
       for (int i = 0; i < ng; ++i) {
-        const int s = i % S;
-        if (!wait_phase(empty0 + 8 * s, ((i / S) & 1) ^ 1, abort_flag, limit)) break;
+        const int s = i % AS;
+        if (!wait_phase(act_empty0 + 8 * s, ((i / AS) & 1) ^ 1, abort_flag, limit)) break;
         const uint32_t full = act_full0 + 8 * s;
         mbar_arrive_expect_tx(full, T::kActStageBytes);
         const uint32_t dst = smem_addr(smem + T::kActOff + s * T::kActStageBytes);
@@ -229,9 +230,9 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
         issued = i + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA's memory goes away
-        for (int i = issued > S ? issued - S : 0; i < issued; ++i) {
+        for (int i = issued > AS ? issued - AS : 0; i < issued; ++i) {
           const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(act_full0 + 8 * (i % S), (i / S) & 1) && global_timer_ns() - t0 < limit) {
+          while (!mbar_try_wait(act_full0 + 8 * (i % AS), (i / AS) & 1) && global_timer_ns() - t0 < limit) {
           }
         }
       }
@@ -267,13 +268,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       // addresses stay below 256 KB).
       const uint64_t desc0 = sw128_kmajor_desc(smem_addr(smem + T::kActOff));
       for (int i = 0; i < ng; ++i) {
-        const int s = i % S;
-        const uint32_t ph = (i / S) & 1;
-        if (!wait_phase(act_full0 + 8 * s, ph, abort_flag, limit)) break;
-        if (!wait_phase(t_ready0 + 8 * s, ph, abort_flag, limit)) break;
+        const int sa = i % AS, st = i % TS;
+        if (!wait_phase(act_full0 + 8 * sa, (i / AS) & 1, abort_flag, limit)) break;
+        if (!wait_phase(t_ready0 + 8 * st, (i / TS) & 1, abort_flag, limit)) break;
         tc_fence_after_sync();
-        const uint64_t desc_s = desc0 + static_cast<uint64_t>((s * T::kActStageBytes) >> 4);
-        const uint32_t a_cols = tmem + T::kACol0 + s * 64;
+        const uint64_t desc_s = desc0 + static_cast<uint64_t>((sa * T::kActStageBytes) >> 4);
+        const uint32_t a_cols = tmem + T::kACol0 + st * 64;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = desc_s + static_cast<uint64_t>(((kk >> 2) * T::kSliceBytes + (kk & 3) * 32) >> 4);
@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
           const uint32_t d = tmem + (step % T::kAccs) * BLOCK_T;
           mma_f16_tmem_a(d, a_cols + kk * 8, bdesc, idesc, step >= T::kAccs ? 1u : 0u);
         }
-        mma_commit(empty0 + 8 * s);
+        mma_commit(act_empty0 + 8 * sa);
+        mma_commit(t_free0 + 8 * st);
       }
       mma_commit(dfull);  // also on abort: lets this thread see its MMAs drain
       if (*abort_flag) {
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     }
     for (int i = half; i < ng; i += 2) {
       const int wj = i / T::kWGroups;  // word stage of this group
-      const int sw = wj % WS, st = i % S;
+      const int sw = wj % WS, st = i % TS;
       uint32_t sc;
       if (staged) {
         sc = sstage[row * ng + i];
@@ -333,7 +334,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
         sq1 = (row_ok && i + 4 < ng) ? __ldg(srow + i + 4) : 0u;
       }
       ok = warp_wait(w_full0 + 8 * sw, (wj / WS) & 1, abort_flag, limit) &&
-           warp_wait(empty0 + 8 * st, ((i / S) & 1) ^ 1, abort_flag, limit);
+           warp_wait(t_free0 + 8 * st, ((i / TS) & 1) ^ 1, abort_flag, limit);
       if (!ok) break;
       tc_fence_after_sync();  // the MMAs that read this TMEM stage are done
       const uint8_t* wstage = smem + T::kWOff + sw * T::kWStageBytes;
