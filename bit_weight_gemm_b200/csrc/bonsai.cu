@@ -251,6 +251,21 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   const int tiles_n = (N + T::kRows - 1) / T::kRows, tiles_m = (M + BLOCK_T - 1) / BLOCK_T;
   const int ksplit = choose_ksplit<MODE, BLOCK_T>(tiles_n * tiles_m, groups);
   if (ksplit > groups) return BONSAI_ERR_SHAPE;
+  // Scale tile by TMA: rows of the scale matrix must be 16-byte multiples
+  // (groups % 8 == 0); the box covers a CTA's groups from an 8-aligned start.
+  CUtensorMap map_s = map_act;  // placeholder when unused
+  int scale_box = 0;
+  if (T::kScaleBytes > 0 && groups % 8 == 0) {
+    const int per_cta = (groups + ksplit - 1) / ksplit;
+    int box = ((per_cta + 7 + 7) / 8) * 8;
+    if (box > groups) box = groups;
+    if (box <= 256 && box * T::kRows * 2 <= T::kScaleBytes) {
+      if (!make_map(&map_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, groups, N, box, T::kRows,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+        return BONSAI_ERR_CUDA;
+      scale_box = box;
+    }
+  }
 
   GemmArgs args;
   args.scales = scales;
@@ -260,6 +275,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   args.K = K;
   args.ksplit = ksplit;
   args.tma_store = tma_store ? 1 : 0;
+  args.scale_box = scale_box;
   args.wait_limit_ns = kDefaultWaitLimitNs;
 
   cudaLaunchConfig_t cfg = {};
@@ -276,7 +292,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
   }
-  if (cudaLaunchKernelEx(&cfg, kernel, map_act, map_w, map_out, args) != cudaSuccess) return BONSAI_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kernel, map_act, map_w, map_out, map_s, args) != cudaSuccess) return BONSAI_ERR_CUDA;
   return launch_status();
 }
 

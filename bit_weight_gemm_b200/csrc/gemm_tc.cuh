@@ -81,7 +81,7 @@ struct GemmTile {
   static constexpr int kWOff = kActStages * kActStageBytes;
   static constexpr int kScaleOff = kWOff + kWStages * kWStageBytes;
   static constexpr int kBarOff = kScaleOff + kScaleBytes;
-  static constexpr int kNumBars = 2 * kActStages + 2 * kTStages + 2 * kWStages + 1;
+  static constexpr int kNumBars = 2 * kActStages + 2 * kTStages + 2 * kWStages + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
   // One CTA per SM: a second CTA could not get its 512 TMEM columns.
@@ -151,13 +151,15 @@ struct GemmArgs {
   int M, N, K;
   int ksplit;     // CTAs along K sharing one tile (the cluster size along z)
   int tma_store;  // 1: write the tile with one TMA store (needs N % 8 == 0)
+  int scale_box;  // > 0: groups per row in the scale TMA box (the tile's scales arrive with one copy)
   uint64_t wait_limit_ns;
 };
 
 template <int MODE, int BLOCK_T>
 __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_w,
-                       const __grid_constant__ CUtensorMap tmap_out, const GemmArgs args) {
+                       const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_s,
+                       const GemmArgs args) {
   using T = GemmTile<MODE, BLOCK_T>;
   constexpr int AS = T::kActStages, TS = T::kTStages, WS = T::kWStages;
   extern __shared__ uint8_t smem_raw[];
@@ -170,6 +172,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
   const uint32_t w_full0 = smem_addr(bars + 2 * AS + 2 * TS);     // TMA bytes of word stage landed
   const uint32_t w_empty0 = smem_addr(bars + 2 * AS + 2 * TS + WS);  // converters read word stage
   const uint32_t dfull = smem_addr(bars + 2 * AS + 2 * TS + 2 * WS);  // accumulator final
+  const uint32_t s_full = smem_addr(bars + 2 * AS + 2 * TS + 2 * WS + 1);  // scale tile landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::kMiscOff + 4);
 
@@ -197,6 +200,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       mbar_init(w_empty0 + 8 * s, T::kConvWarps);  // every converter warp reads each full stage
     }
     mbar_init(dfull, 1);
+    mbar_init(s_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -204,6 +208,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     tma_prefetch_map(&tmap_act);
     tma_prefetch_map(&tmap_w);
     tma_prefetch_map(&tmap_out);
+    if (args.scale_box > 0) tma_prefetch_map(&tmap_s);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), T::kTmemCols);
@@ -240,6 +245,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------ packed-word producer
     if (elect_one()) {
+      if (args.scale_box > 0) {
+        // The tile's scales: 128 rows x scale_box groups from an 8-aligned
+        // group column (TMA needs 16-byte aligned starts).
+        mbar_arrive_expect_tx(s_full, static_cast<uint32_t>(args.scale_box) * T::kRows * 2);
+        tma_load_2d(smem_addr(smem + T::kScaleOff), &tmap_s, s_full, g_begin & ~7, n0);
+      }
       int issued = 0;
       const int nw = (ng + T::kWGroups - 1) / T::kWGroups;
       for (int i = 0; i < nw; ++i) {
@@ -302,32 +313,44 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint16_t* srow = args.scales + static_cast<size_t>(n) * groups + g_begin;
     const bool row_ok = n < args.N;
-    // Scales: all of the tile's at once into shared memory when they fit
-    // (their loads overlap the first packed-word loads), else two groups
-    // ahead in registers.
-    const bool staged = T::kScaleBytes > 0 && T::kRows * ng * 2 <= T::kScaleBytes;
+    // Scales: the whole tile's in shared memory when they fit, by one TMA
+    // (scale_box > 0) or by batched loads; else two groups ahead in registers.
+    const bool by_tma = args.scale_box > 0;
+    const bool staged = by_tma || (T::kScaleBytes > 0 && T::kRows * ng * 2 <= T::kScaleBytes);
+    const int s_stride = by_tma ? args.scale_box : ng;  // groups per row in the staged tile
+    const int s_first = by_tma ? g_begin - (g_begin & ~7) : 0;
     uint16_t* sstage = reinterpret_cast<uint16_t*>(smem + T::kScaleOff);
-    if (staged) {
+    if (!by_tma && staged) {
       const int ct = threadIdx.x - 96;  // 0 .. 255 over the converter warps
-      for (int e = ct; e < T::kRows * ng; e += 32 * T::kConvWarps) {
-        const int r = e / ng, g = e - (e / ng) * ng;
-        sstage[e] = (n0 + r < args.N) ? __ldg(args.scales + static_cast<size_t>(n0 + r) * groups + g_begin + g)
-                                      : uint16_t(0);
+      constexpr int kBatch = 8;         // independent loads in flight per thread
+      for (int e0 = ct; e0 < T::kRows * ng; e0 += kBatch * 32 * T::kConvWarps) {
+        uint16_t v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int e = e0 + u * 32 * T::kConvWarps;
+          const int r = e / ng, g = e - (e / ng) * ng;
+          v[u] = (e < T::kRows * ng && n0 + r < args.N)
+                     ? __ldg(args.scales + static_cast<size_t>(n0 + r) * groups + g_begin + g)
+                     : uint16_t(0);
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (e0 + u * 32 * T::kConvWarps < T::kRows * ng) sstage[e0 + u * 32 * T::kConvWarps] = v[u];
       }
       named_barrier_sync(2, 32 * T::kConvWarps);
     }
     uint32_t sq0 = 0, sq1 = 0;
-    bool ok = true;
+    bool ok = !by_tma || warp_wait(s_full, 0, abort_flag, limit);
     if (!staged) {
       sq0 = (row_ok && half < ng) ? __ldg(srow + half) : 0u;
       sq1 = (row_ok && half + 2 < ng) ? __ldg(srow + half + 2) : 0u;
     }
-    for (int i = half; i < ng; i += 2) {
+    for (int i = half; ok && i < ng; i += 2) {
       const int wj = i / T::kWGroups;  // word stage of this group
       const int sw = wj % WS, st = i % TS;
       uint32_t sc;
       if (staged) {
-        sc = sstage[row * ng + i];
+        sc = sstage[row * s_stride + s_first + i];
       } else {
         sc = sq0;
         sq0 = sq1;
