@@ -13,8 +13,8 @@
 //                        with 128-byte swizzling, so that the converters'
 //                        16-byte reads are free of bank conflicts and each
 //                        request moves a whole 128-byte line.
-//   TMEM ring  (warps 3-10, two per TMEM lane quadrant, taking alternate
-//                        groups) converters: each thread owns one weight row,
+//   TMEM ring  (warps 3-18, four per TMEM lane quadrant, taking groups in
+//                        turn) converters: each thread owns one weight row,
 //                        turns the group's words into exact FP16 products
 //                        (binary: sign bit over s; ternary: the shifted 2-bit
 //                        field is 2t, times s) and writes them to a TMEM
@@ -69,7 +69,10 @@ struct GemmTile {
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
   static constexpr int kTStages = BLOCK_T >= 256 ? 3 : 4;  // TMEM stages of converted weights, 64 columns each
-  static constexpr int kConvWarps = 8;
+  static constexpr int kConvWarps = 16;           // four per TMEM lane quadrant
+  static constexpr int kWarpsPerQuad = kConvWarps / 4;
+  // Epilogue: the quadrant's warps split the token columns, 8 at least each.
+  static constexpr int kEpiWarpsPerQuad = BLOCK_T / 8 < kWarpsPerQuad ? BLOCK_T / 8 : kWarpsPerQuad;
   static constexpr int kThreads = 32 * (3 + kConvWarps);
   // Successive MMAs rotate over kAccs accumulators [a*BLOCK_T, (a+1)*BLOCK_T):
   // with narrow tiles an MMA is a few cycles of work, so a chain of MMAs into
@@ -304,10 +307,10 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------ converters, epilogue
-    // The two warps of a TMEM lane quadrant take alternate groups, so that
-    // one's barrier waits overlap the other's conversion.
+    // The warps of a TMEM lane quadrant take groups in turn, so that one's
+    // barrier waits and latencies overlap the others' conversion.
     const int quad = warp & 3;  // a warp may only touch TMEM lanes 32*(warp%4) .. +31
-    const int half = (warp - 3) >> 2;
+    const int turn = (warp - 3) >> 2;  // 0 .. kWarpsPerQuad-1
     const int row = quad * 32 + lane;
     const int n = n0 + row;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
@@ -321,7 +324,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     const int s_first = by_tma ? g_begin - (g_begin & ~7) : 0;
     uint16_t* sstage = reinterpret_cast<uint16_t*>(smem + T::kScaleOff);
     if (!by_tma && staged) {
-      const int ct = threadIdx.x - 96;  // 0 .. 255 over the converter warps
+      const int ct = threadIdx.x - 96;  // 0 .. 32 * kConvWarps - 1 over the converter warps
       constexpr int kBatch = 8;         // independent loads in flight per thread
       for (int e0 = ct; e0 < T::kRows * ng; e0 += kBatch * 32 * T::kConvWarps) {
         uint16_t v[kBatch];
@@ -341,11 +344,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     }
     uint32_t sq0 = 0, sq1 = 0;
     bool ok = !by_tma || warp_wait(s_full, 0, abort_flag, limit);
+    constexpr int kStep = T::kWarpsPerQuad;
     if (!staged) {
-      sq0 = (row_ok && half < ng) ? __ldg(srow + half) : 0u;
-      sq1 = (row_ok && half + 2 < ng) ? __ldg(srow + half + 2) : 0u;
+      sq0 = (row_ok && turn < ng) ? __ldg(srow + turn) : 0u;
+      sq1 = (row_ok && turn + kStep < ng) ? __ldg(srow + turn + kStep) : 0u;
     }
-    for (int i = half; ok && i < ng; i += 2) {
+    for (int i = turn; ok && i < ng; i += kStep) {
       const int wj = i / T::kWGroups;  // word stage of this group
       const int sw = wj % WS, st = i % TS;
       uint32_t sc;
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       } else {
         sc = sq0;
         sq0 = sq1;
-        sq1 = (row_ok && i + 4 < ng) ? __ldg(srow + i + 4) : 0u;
+        sq1 = (row_ok && i + 2 * kStep < ng) ? __ldg(srow + i + 2 * kStep) : 0u;
       }
       ok = warp_wait(w_full0 + 8 * sw, (wj / WS) & 1, abort_flag, limit) &&
            warp_wait(t_free0 + 8 * st, ((i / TS) & 1) ^ 1, abort_flag, limit);
@@ -386,7 +390,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       __syncwarp();
       // Release the word stage after this warp's last group in it.
       const int stage_end = (wj + 1) * T::kWGroups < ng ? (wj + 1) * T::kWGroups : ng;
-      if (lane == 0 && i + 2 >= stage_end) mbar_arrive(w_empty0 + 8 * sw);
+      if (lane == 0 && i + kStep >= stage_end) mbar_arrive(w_empty0 + 8 * sw);
       convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
       tmem_store_wait();
       tc_fence_before_sync();
@@ -395,14 +399,15 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     }
     if (ok) ok = warp_wait(dfull, 0, abort_flag, limit);
     if (ok) tc_fence_after_sync();
-    constexpr int kHalfCols = BLOCK_T / 2;
-    const int c_begin = half * kHalfCols;
+    constexpr int kEpiCols = BLOCK_T / T::kEpiWarpsPerQuad;  // token columns per epilogue warp
+    const bool epi = turn < T::kEpiWarpsPerQuad;
+    const int c_begin = turn * kEpiCols;
     if (args.ksplit == 1) {
       // FP16 tile [BLOCK_T tokens][128 rows] in the (now idle) act ring.
       uint16_t* tile = reinterpret_cast<uint16_t*>(smem + T::kActOff);
-      if (ok) {
+      if (ok && epi) {
 #pragma unroll 1
-        for (int c = 0; c < kHalfCols; c += 8) {
+        for (int c = 0; c < kEpiCols; c += 8) {
           float acc[8];
           sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, acc);
 #pragma unroll
@@ -422,18 +427,18 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
             bulk_wait_group_read0();
           }
         } else {
-          const int ct = threadIdx.x - 96;  // 0 .. 255 over the converter warps
+          const int ct = threadIdx.x - 96;  // 0 .. 32 * kConvWarps - 1 over the converter warps
           for (int e = ct; e < BLOCK_T * T::kRows; e += 32 * T::kConvWarps) {
             const int m = m0 + e / T::kRows, nn = n0 + e % T::kRows;
             if (m < args.M && nn < args.N) args.out[static_cast<size_t>(m) * args.N + nn] = tile[e];
           }
         }
       }
-    } else if (ok) {
+    } else if (ok && epi) {
       // FP32 partial [BLOCK_T tokens][128 rows] in the act ring.
       float* part = reinterpret_cast<float*>(smem + T::kActOff);
 #pragma unroll 1
-      for (int c = 0; c < kHalfCols; c += 8) {
+      for (int c = 0; c < kEpiCols; c += 8) {
         float acc[8];
         sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, acc);
 #pragma unroll
