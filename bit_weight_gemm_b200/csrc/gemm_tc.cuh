@@ -68,7 +68,7 @@ struct GemmTile {
   static constexpr int kWStages = BLOCK_T >= 256 ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
-  static constexpr int kTStages = BLOCK_T >= 256 ? 3 : 4;  // TMEM stages of converted weights, 64 columns each
+  static constexpr int kTStages = 4;  // TMEM stages of converted weights, 64 columns each
   static constexpr int kConvWarps = 16;           // four per TMEM lane quadrant
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
   // Epilogue: the quadrant's warps split the token columns, 8 at least each.
@@ -94,6 +94,10 @@ struct GemmTile {
   static_assert(BLOCK_T % 16 == 0 && BLOCK_T >= 16 && BLOCK_T <= 256, "MMA N for M=128");
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kTmemCols == 512, "one CTA per SM holds all of tensor memory");
+  // A converter warp takes every kWarpsPerQuad-th group, so it can wait on a
+  // TMEM stage at most one use ahead of the MMAs only if there are at least
+  // that many stages; with fewer, a parity wait could match an older phase.
+  static_assert(kWarpsPerQuad <= kTStages, "converter warps per quadrant <= TMEM stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(BLOCK_T * kRows * 2 <= kActStages * kActStageBytes, "output tile fits the act ring");
   static_assert(kRows * BLOCK_T * 4 <= kActStages * kActStageBytes, "partial fits the act ring");
