@@ -68,11 +68,6 @@ struct GemmTile {
   static constexpr int kWStages = BLOCK_T >= 256 ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
-  // TMEM stages of converted weights, 64 columns each: all that is left
-  // after the accumulators.  A stage is reused only after the MMAs that read
-  // it completed, so the number of stages is the number of groups in flight
-  // between the converters and the tensor core.
-  static constexpr int kTStages = (512 - kACol0) / 64;
   static constexpr int kConvWarps = 16;           // four per TMEM lane quadrant
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
   // Epilogue: the quadrant's warps split the token columns, 8 at least each.
@@ -83,6 +78,11 @@ struct GemmTile {
   // one accumulator would run at the accumulate latency instead.
   static constexpr int kAccs = BLOCK_T <= 32 ? 2 : 1;
   static constexpr int kACol0 = kAccs * BLOCK_T < 64 ? 64 : kAccs * BLOCK_T;  // converted-weight stages follow
+  // TMEM stages of converted weights, 64 columns each: all that is left
+  // after the accumulators.  A stage is reused only after the MMAs that read
+  // it completed, so the number of stages is the number of groups in flight
+  // between the converters and the tensor core.
+  static constexpr int kTStages = (512 - kACol0) / 64;
   static constexpr int kTmemCols = pow2_at_least(kACol0 + kTStages * 64);
   static constexpr int kActOff = 0;
   static constexpr int kWOff = kActStages * kActStageBytes;
