@@ -131,12 +131,17 @@ __device__ __forceinline__ void convert_group(const uint32_t* words, uint32_t s2
   }
 }
 
-// A wait the whole warp agrees on: every lane waits, and the warp goes on
-// only if all lanes saw the phase complete.
+// A wait for the whole warp: lane 0 alone polls the barrier (32 lanes
+// polling one mbarrier would queue on the SM's barrier unit and slow every
+// other warp's barrier operations), then shares the outcome; __syncwarp
+// orders the other lanes' later reads after lane 0's acquire.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t limit_ns) {
-  const bool ok = wait_phase(bar, parity, abort_flag, limit_ns);
-  return __all_sync(0xffffffffu, ok);
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, abort_flag, limit_ns);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
 }
 
 // Reads 8 columns of this thread's lane from each of the NACC accumulators
