@@ -131,17 +131,12 @@ __device__ __forceinline__ void convert_group(const uint32_t* words, uint32_t s2
   }
 }
 
-// A wait for the whole warp: lane 0 alone polls the barrier (32 lanes
-// polling one mbarrier would queue on the SM's barrier unit and slow every
-// other warp's barrier operations), then shares the outcome; __syncwarp
-// orders the other lanes' later reads after lane 0's acquire.
+// A wait the whole warp agrees on: every lane waits, and the warp goes on
+// only if all lanes saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t limit_ns) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, abort_flag, limit_ns);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  __syncwarp();
-  return ok;
+  const bool ok = wait_phase(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Reads 8 columns of this thread's lane from each of the NACC accumulators
@@ -294,10 +289,19 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       // offset >> 4 to the start-address field (no carry: shared memory
       // addresses stay below 256 KB).
       const uint64_t desc0 = sw128_kmajor_desc(smem_addr(smem + T::kActOff));
+      // Group i's stages are released (tcgen05.commit) only after the waits
+      // for group i+1: a barrier wait issued after a commit would not return
+      // before that commit's MMAs complete, which would drain the tensor core
+      // between groups.
+      int prev_sa = -1, prev_st = -1;
       for (int i = 0; i < ng; ++i) {
         const int sa = i % AS, st = i % TS;
         if (!wait_phase(act_full0 + 8 * sa, (i / AS) & 1, abort_flag, limit)) break;
         if (!wait_phase(t_ready0 + 8 * st, (i / TS) & 1, abort_flag, limit)) break;
+        if (prev_sa >= 0) {
+          mma_commit(act_empty0 + 8 * prev_sa);
+          mma_commit(t_free0 + 8 * prev_st);
+        }
         tc_fence_after_sync();
         const uint64_t desc_s = desc0 + static_cast<uint64_t>((sa * T::kActStageBytes) >> 4);
         const uint32_t a_cols = tmem + T::kACol0 + st * 64;
@@ -308,8 +312,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
           const uint32_t d = tmem + (step % T::kAccs) * BLOCK_T;
           mma_f16_tmem_a(d, a_cols + kk * 8, bdesc, idesc, step >= T::kAccs ? 1u : 0u);
         }
-        mma_commit(act_empty0 + 8 * sa);
-        mma_commit(t_free0 + 8 * st);
+        prev_sa = sa;
+        prev_st = st;
+      }
+      if (prev_sa >= 0) {
+        mma_commit(act_empty0 + 8 * prev_sa);
+        mma_commit(t_free0 + 8 * prev_st);
       }
       mma_commit(dfull);  // also on abort: lets this thread see its MMAs drain
       if (*abort_flag) {
