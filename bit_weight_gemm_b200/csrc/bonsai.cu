@@ -170,9 +170,9 @@ int sm_count() {
 }
 
 // Clusters of `ksplit` CTAs that can be resident at once (0 if unknown).
-template <int MODE, int BLOCK_T>
+template <int MODE, int BLOCK_T, int OCC>
 int resident_clusters(int ksplit) {
-  using T = GemmTile<MODE, BLOCK_T>;
+  using T = GemmTile<MODE, BLOCK_T, OCC>;
   static std::mutex mu;
   static int cache[9] = {0};
   std::lock_guard<std::mutex> lock(mu);
@@ -190,7 +190,7 @@ int resident_clusters(int ksplit) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, lowbit_gemm_kernel<MODE, BLOCK_T>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, lowbit_gemm_kernel<MODE, BLOCK_T, OCC>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       n = -1;
     }
@@ -201,14 +201,14 @@ int resident_clusters(int ksplit) {
 
 // Split K over a cluster when the tiles alone leave SMs idle: pick the split
 // that minimises waves x groups per CTA.
-template <int MODE, int BLOCK_T>
+template <int MODE, int BLOCK_T, int OCC>
 int choose_ksplit(int tiles, int groups) {
-  const int sms = sm_count();
+  const int sms = sm_count() * OCC;
   if (tiles >= sms) return 1;
   int best = 1;
   double best_cost = 1e30;
   for (int ks = 1; ks <= 8 && ks <= groups; ++ks) {
-    const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T>(ks);
+    const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T, OCC>(ks);
     if (per_wave <= 0) continue;
     const int waves = (tiles + per_wave - 1) / per_wave;
     const double cost = static_cast<double>(waves) * ((groups + ks - 1) / ks) + 0.25 * ks;  // small cost per split
@@ -220,11 +220,11 @@ int choose_ksplit(int tiles, int groups) {
   return best;
 }
 
-template <int MODE, int BLOCK_T>
+template <int MODE, int BLOCK_T, int OCC>
 int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, uint16_t* out,
                 cudaStream_t stream) {
-  using T = GemmTile<MODE, BLOCK_T>;
-  auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T>;
+  using T = GemmTile<MODE, BLOCK_T, OCC>;
+  auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T, OCC>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -249,7 +249,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   }
   const int groups = K / kGroup;
   const int tiles_n = (N + T::kRows - 1) / T::kRows, tiles_m = (M + BLOCK_T - 1) / BLOCK_T;
-  const int ksplit = choose_ksplit<MODE, BLOCK_T>(tiles_n * tiles_m, groups);
+  const int ksplit = choose_ksplit<MODE, BLOCK_T, OCC>(tiles_n * tiles_m, groups);
   if (ksplit > groups) return BONSAI_ERR_SHAPE;
   // Scale tile by TMA: rows of the scale matrix must be 16-byte multiples
   // (groups % 8 == 0); the box covers a CTA's groups from an 8-aligned start.
@@ -296,34 +296,43 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   return launch_status();
 }
 
+// More than 128 tokens: 128-token tiles, two CTAs per SM (one CTA's
+// prologue and epilogue overlap the other's MMAs).
+#ifndef BONSAI_LARGE_TILE
+#define BONSAI_LARGE_TILE 128
+#define BONSAI_LARGE_OCC 2
+#endif
+constexpr int kLargeTile = BONSAI_LARGE_TILE;
+constexpr int kLargeOcc = BONSAI_LARGE_OCC;
+
 struct Plan {
   int block_t, ksplit, ctas;
 };
 
-template <int MODE, int BLOCK_T>
+template <int MODE, int BLOCK_T, int OCC>
 Plan plan_for(int M, int N, int K) {
   const int tiles = ((N + 127) / 128) * ((M + BLOCK_T - 1) / BLOCK_T);
-  const int ks = choose_ksplit<MODE, BLOCK_T>(tiles, K / kGroup);
+  const int ks = choose_ksplit<MODE, BLOCK_T, OCC>(tiles, K / kGroup);
   return Plan{BLOCK_T, ks, tiles * ks};
 }
 
 template <int MODE>
 Plan plan_gemm(int M, int N, int K) {
-  if (M <= 16) return plan_for<MODE, 16>(M, N, K);
-  if (M <= 32) return plan_for<MODE, 32>(M, N, K);
-  if (M <= 64) return plan_for<MODE, 64>(M, N, K);
-  if (M <= 128) return plan_for<MODE, 128>(M, N, K);
-  return plan_for<MODE, 256>(M, N, K);
+  if (M <= 16) return plan_for<MODE, 16, 1>(M, N, K);
+  if (M <= 32) return plan_for<MODE, 32, 1>(M, N, K);
+  if (M <= 64) return plan_for<MODE, 64, 1>(M, N, K);
+  if (M <= 128) return plan_for<MODE, 128, 1>(M, N, K);
+  return plan_for<MODE, kLargeTile, kLargeOcc>(M, N, K);
 }
 
 template <int MODE>
 int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
                   uint16_t* out, cudaStream_t stream) {
-  if (M <= 16) return launch_gemm<MODE, 16>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 32) return launch_gemm<MODE, 32>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 64) return launch_gemm<MODE, 64>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 128) return launch_gemm<MODE, 128>(A, packed, scales, M, N, K, out, stream);
-  return launch_gemm<MODE, 256>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 16) return launch_gemm<MODE, 16, 1>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 32) return launch_gemm<MODE, 32, 1>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 64) return launch_gemm<MODE, 64, 1>(A, packed, scales, M, N, K, out, stream);
+  if (M <= 128) return launch_gemm<MODE, 128, 1>(A, packed, scales, M, N, K, out, stream);
+  return launch_gemm<MODE, kLargeTile, kLargeOcc>(A, packed, scales, M, N, K, out, stream);
 }
 
 }  // namespace

@@ -50,7 +50,11 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
   return p;
 }
 
-template <int MODE, int BLOCK_T>
+// OCC = CTAs per SM.  OCC 1: a CTA owns all 512 TMEM columns and most of
+// shared memory.  OCC 2 (tiles of at most 128 tokens): two CTAs share an SM,
+// 256 TMEM columns and ~110 KB of shared memory each, so that one CTA's
+// prologue and epilogue overlap the other's MMAs.
+template <int MODE, int BLOCK_T, int OCC = 1>
 struct GemmTile {
   static constexpr int kRows = 128;  // weight rows per tile (MMA M)
   static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : 8;
@@ -58,17 +62,19 @@ struct GemmTile {
   static constexpr int kActStageBytes = 2 * kSliceBytes;  // 128 K per stage
   // Activation stages: as many as fit next to the word ring and the scales,
   // so that narrow tiles keep a split-K CTA's whole K range in flight.
-  static constexpr int kActStages = BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : (96 * 1024) / kActStageBytes);
+  static constexpr int kActStages =
+      OCC == 2 ? (64 * 1024) / kActStageBytes
+               : (BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : (96 * 1024) / kActStageBytes));
   // A word stage is 128 bytes of every row: 4 ternary or 8 binary groups,
   // one TMA box with 128-byte swizzling.
   static constexpr int kWGroups = 32 / kWordsPerGroup;
   static constexpr int kWStageBytes = kRows * 128;
   // Small token tiles are bandwidth-bound: enough word stages to keep every
   // load of a split-K CTA in flight at once.
-  static constexpr int kWStages = BLOCK_T >= 256 ? 2 : 4;
+  static constexpr int kWStages = (OCC == 2 || BLOCK_T >= 256) ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
-  static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
-  static constexpr int kConvWarps = 16;           // four per TMEM lane quadrant
+  static constexpr int kScaleBytes = (OCC == 2 || BLOCK_T >= 256) ? 0 : 32768;
+  static constexpr int kConvWarps = OCC == 2 ? 8 : 16;  // 2 or 4 per TMEM lane quadrant
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
   // Epilogue: the quadrant's warps split the token columns, 8 at least each.
   static constexpr int kEpiWarpsPerQuad = BLOCK_T / 8 < kWarpsPerQuad ? BLOCK_T / 8 : kWarpsPerQuad;
@@ -82,8 +88,8 @@ struct GemmTile {
   // after the accumulators.  A stage is reused only after the MMAs that read
   // it completed, so the number of stages is the number of groups in flight
   // between the converters and the tensor core.
-  static constexpr int kTStages = (512 - kACol0) / 64;
-  static constexpr int kTmemCols = pow2_at_least(kACol0 + kTStages * 64);
+  static constexpr int kTmemCols = 512 / OCC;
+  static constexpr int kTStages = (kTmemCols - kACol0) / 64;
   static constexpr int kActOff = 0;
   static constexpr int kWOff = kActStages * kActStageBytes;
   static constexpr int kScaleOff = kWOff + kWStages * kWStageBytes;
@@ -91,18 +97,21 @@ struct GemmTile {
   static constexpr int kNumBars = 2 * kActStages + 2 * kTStages + 2 * kWStages + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
-  // One CTA per SM: a second CTA could not get its 512 TMEM columns.
-  static constexpr int kSmemBytes = kSmemNeeded > 116 * 1024 ? kSmemNeeded : 116 * 1024;
+  // OCC 1: a second CTA could not get its 512 TMEM columns, so shared memory
+  // keeps it off the SM.
+  static constexpr int kSmemBytes = (OCC == 1 && kSmemNeeded < 116 * 1024) ? 116 * 1024 : kSmemNeeded;
 
   static constexpr float kOutScale = MODE == BONSAI_BINARY ? 1.0f : 0.5f;
   static_assert(BLOCK_T % 16 == 0 && BLOCK_T >= 16 && BLOCK_T <= 256, "MMA N for M=128");
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
-  static_assert(kTmemCols == 512, "one CTA per SM holds all of tensor memory");
+  static_assert(OCC == 1 || OCC == 2, "one or two CTAs per SM");
+  static_assert(kACol0 + kTStages * 64 <= kTmemCols && kTStages >= 2, "TMEM budget");
   // A converter warp takes every kWarpsPerQuad-th group, so it can wait on a
   // TMEM stage at most one use ahead of the MMAs only if there are at least
   // that many stages; with fewer, a parity wait could match an older phase.
   static_assert(kWarpsPerQuad <= kTStages, "converter warps per quadrant <= TMEM stages");
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+  static_assert(kSmemBytes <= (OCC == 1 ? 227 * 1024 : 113 * 1024), "shared memory per CTA");
+  static_assert(kActStages >= 2, "activation ring depth");
   static_assert(BLOCK_T * kRows * 2 <= kActStages * kActStageBytes, "output tile fits the act ring");
   static_assert(kRows * BLOCK_T * 4 <= kActStages * kActStageBytes, "partial fits the act ring");
 };
@@ -166,12 +175,12 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
 };
 
-template <int MODE, int BLOCK_T>
-__global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
+template <int MODE, int BLOCK_T, int OCC>
+__global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_s,
                        const GemmArgs args) {
-  using T = GemmTile<MODE, BLOCK_T>;
+  using T = GemmTile<MODE, BLOCK_T, OCC>;
   constexpr int AS = T::kActStages, TS = T::kTStages, WS = T::kWStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

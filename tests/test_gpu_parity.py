@@ -189,7 +189,8 @@ def test_gemm_full_size_sampled(oracle_mod, problem):
 
 def test_plans_cover_both_epilogues():
     big = bw.gemm_plan(4608, 9216, 3072, "ternary")
-    assert big == {"block_t": 256, "ksplit": 1, "ctas": 72 * 18}
+    assert big["ksplit"] == 1 and big["block_t"] in (128, 256)
+    assert big["ctas"] == 72 * (4608 // big["block_t"])
     for M, N, K in [(16, 3072, 9216), (16, 9216, 3072), (16, 256, 4096), (40, 384, 2048)]:
         p = bw.gemm_plan(M, N, K, "ternary")
         assert 1 < p["ksplit"] <= 8 and p["ctas"] % p["ksplit"] == 0, (M, N, K, p)
