@@ -346,6 +346,9 @@ def run_bonsai(args):
     small = None
     if not args.no_extras or args.small_only:
         small = time_small(torch, bw, SMALL, args, dist, peaks, peaks_kind)
+    stack = None
+    if not args.no_extras and not args.small_only:
+        stack = [time_stack(torch, bw, m, "ternary", 20, 3) for m in (4608, 1024)]
 
     if dist is not None:
         dist.barrier()
@@ -371,6 +374,7 @@ def run_bonsai(args):
                 "e2e": result["e2e"],
                 "cpu_baseline": cpu,
                 "small_m": small,
+                "stack": stack,
             }
             print(json.dumps(line), flush=True)
     if dist is not None:
@@ -437,6 +441,52 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
                          "frac": achieved / peak, "traffic": ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}"),
                          "algorithmic_bytes_per_launch": nbytes, "peak_source": f"{peaks_kind} hbm copy"},
             "gpu_launches": steps}
+
+
+def time_stack(torch, bw, M, mode, steps, warmup, seed=2000):
+    """One denoise step of the 25-block MMDiT stack (80 launches = 100 linears,
+    Q|K|V stacked): every layer has its own weight buffers (cloned from one
+    seeded set per distinct shape), the step is captured as one CUDA graph."""
+    layers = workloads.mmdit_stack_layers()
+    shapes = sorted({(n, k) for _, n, k in layers})
+    base = {}
+    for j, (n, k) in enumerate(shapes):
+        d = workloads.make(mode=mode, M=1, N=n, K=k, seed=seed + j)
+        packed = bw.pack(torch.from_numpy(d["codes"]).cuda(), mode)
+        scales = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+        base[(n, k)] = (packed, scales)
+    weights = [tuple(t.clone() for t in base[(n, k)]) for _, n, k in layers]
+    rng = np.random.default_rng(seed)
+    acts = {k: torch.from_numpy(workloads.activations(rng, M, k).view(np.int16)).view(torch.float16).cuda()
+            for k in {k for _, _, k in layers}}
+    outs = {n: torch.empty((M, n), dtype=torch.float16, device="cuda") for n in {n for _, n, _ in layers}}
+
+    def step():
+        for (name, n, k), (packed, scales) in zip(layers, weights):
+            bw.lowbit_gemm(acts[k], packed, scales, mode, out=outs[n])
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        graph.replay()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    total_flops = sum(2 * M * n * k for _, n, k in layers)
+    wbytes = sum(n * k // (8 if mode == "binary" else 4) + 2 * n * (k // 128) for _, n, k in layers)
+    del graph
+    return {"M": M, "mode": mode, "launches": len(layers), "ms_per_denoise_step": ms,
+            "tflops": total_flops / (ms * 1e-3) / 1e12, "weight_bytes": wbytes,
+            "weight_gbs": wbytes / (ms * 1e-3) / 1e9}
 
 
 def main():

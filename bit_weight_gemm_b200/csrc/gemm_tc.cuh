@@ -298,35 +298,31 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
       // offset >> 4 to the start-address field (no carry: shared memory
       // addresses stay below 256 KB).
       const uint64_t desc0 = sw128_kmajor_desc(smem_addr(smem + T::kActOff));
-      // Group i's stages are released (tcgen05.commit) only after the waits
-      // for group i+1: a barrier wait issued after a commit would not return
-      // before that commit's MMAs complete, which would drain the tensor core
-      // between groups.
-      int prev_sa = -1, prev_st = -1;
-      for (int i = 0; i < ng; ++i) {
+      // Software-pipelined: the waits for group i+1 sit between group i's
+      // first six and last two MMAs, so the tensor core still has queued
+      // work while this thread polls the barriers.
+      bool ready = ng > 0 && wait_phase(act_full0, 0, abort_flag, limit) && wait_phase(t_ready0, 0, abort_flag, limit);
+      for (int i = 0; ready && i < ng; ++i) {
         const int sa = i % AS, st = i % TS;
-        if (!wait_phase(act_full0 + 8 * sa, (i / AS) & 1, abort_flag, limit)) break;
-        if (!wait_phase(t_ready0 + 8 * st, (i / TS) & 1, abort_flag, limit)) break;
-        if (prev_sa >= 0) {
-          mma_commit(act_empty0 + 8 * prev_sa);
-          mma_commit(t_free0 + 8 * prev_st);
-        }
         tc_fence_after_sync();
         const uint64_t desc_s = desc0 + static_cast<uint64_t>((sa * T::kActStageBytes) >> 4);
         const uint32_t a_cols = tmem + T::kACol0 + st * 64;
+        bool next_ready = true;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+          if (kk == 6 && i + 1 < ng) {
+            const int na = (i + 1) % AS, nt = (i + 1) % TS;
+            next_ready = wait_phase(act_full0 + 8 * na, ((i + 1) / AS) & 1, abort_flag, limit) &&
+                         wait_phase(t_ready0 + 8 * nt, ((i + 1) / TS) & 1, abort_flag, limit);
+          }
           const uint64_t bdesc = desc_s + static_cast<uint64_t>(((kk >> 2) * T::kSliceBytes + (kk & 3) * 32) >> 4);
           const int step = i * 8 + kk;
           const uint32_t d = tmem + (step % T::kAccs) * BLOCK_T;
           mma_f16_tmem_a(d, a_cols + kk * 8, bdesc, idesc, step >= T::kAccs ? 1u : 0u);
         }
-        prev_sa = sa;
-        prev_st = st;
-      }
-      if (prev_sa >= 0) {
-        mma_commit(act_empty0 + 8 * prev_sa);
-        mma_commit(t_free0 + 8 * prev_st);
+        mma_commit(act_empty0 + 8 * sa);
+        mma_commit(t_free0 + 8 * st);
+        ready = next_ready;
       }
       mma_commit(dfull);  // also on abort: lets this thread see its MMAs drain
       if (*abort_flag) {
