@@ -78,11 +78,18 @@ struct GemmTile {
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
   // Epilogue: the quadrant's warps split the token columns, 8 at least each.
   static constexpr int kEpiWarpsPerQuad = BLOCK_T / 8 < kWarpsPerQuad ? BLOCK_T / 8 : kWarpsPerQuad;
-  static constexpr int kThreads = 32 * (3 + kConvWarps);
+  // Two MMA-issuing threads (alternate groups, separate accumulators) and
+  // two activation producers for tiles of up to 128 tokens, where one thread
+  // issuing every MMA and polling every barrier is the serial limit.  A
+  // 256-token accumulator fills half of TMEM, so those tiles keep one.
+  static constexpr int kMmaThreads = (OCC == 1 && BLOCK_T <= 128) ? 2 : 1;
+  static constexpr int kActWarpB = 3 + kConvWarps;  // second activation producer
+  static constexpr int kMmaWarpB = 4 + kConvWarps;  // second MMA issuer (idle when kMmaThreads == 1)
+  static constexpr int kThreads = 32 * (5 + kConvWarps);
   // Successive MMAs rotate over kAccs accumulators [a*BLOCK_T, (a+1)*BLOCK_T):
   // with narrow tiles an MMA is a few cycles of work, so a chain of MMAs into
   // one accumulator would run at the accumulate latency instead.
-  static constexpr int kAccs = BLOCK_T <= 32 ? 2 : 1;
+  static constexpr int kAccs = (kMmaThreads == 2 || BLOCK_T <= 32) ? 2 : 1;
   static constexpr int kACol0 = kAccs * BLOCK_T < 64 ? 64 : kAccs * BLOCK_T;  // converted-weight stages follow
   // TMEM stages of converted weights, 64 columns each: all that is left
   // after the accumulators.  A stage is reused only after the MMAs that read
@@ -149,9 +156,10 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // Reads 8 columns of this thread's lane from each of the NACC accumulators
-// (NACC * BLOCK_T columns apart) and adds them in a fixed order.
+// (BLOCK_T columns apart) and adds the first `used` of them in a fixed order
+// (an accumulator no MMA wrote holds nothing meaningful).
 template <int NACC, int BLOCK_T>
-__device__ __forceinline__ void sum_accumulators(uint32_t taddr, float* acc) {
+__device__ __forceinline__ void sum_accumulators(uint32_t taddr, int used, float* acc) {
   uint32_t v[NACC][8];
 #pragma unroll
   for (int a = 0; a < NACC; ++a) tmem_load_8(taddr + a * BLOCK_T, v[a]);
@@ -160,7 +168,8 @@ __device__ __forceinline__ void sum_accumulators(uint32_t taddr, float* acc) {
   for (int j = 0; j < 8; ++j) {
     float x = __uint_as_float(v[0][j]);
 #pragma unroll
-    for (int a = 1; a < NACC; ++a) x += __uint_as_float(v[a][j]);
+    for (int a = 1; a < NACC; ++a)
+      if (a < used) x += __uint_as_float(v[a][j]);
     acc[j] = x;
   }
 }
@@ -219,7 +228,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
       mbar_init(w_full0 + 8 * s, 1);
       mbar_init(w_empty0 + 8 * s, T::kConvWarps);  // every converter warp reads each full stage
     }
-    mbar_init(dfull, 1);
+    mbar_init(dfull, T::kMmaThreads);
     mbar_init(s_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -239,11 +248,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------- activation producer
+  if (warp == 0 || warp == T::kActWarpB) {
+    // ------------------------------------- activation producers (2, alternate groups)
+    const int first = warp == 0 ? 0 : 1;
     if (elect_one()) {
       int issued = 0;
-      for (int i = 0; i < ng; ++i) {
+      for (int i = first; i < ng; i += 2) {
         const int s = i % AS;
         if (!wait_phase(act_empty0 + 8 * s, ((i / AS) & 1) ^ 1, abort_flag, limit)) break;
         const uint32_t full = act_full0 + 8 * s;
@@ -255,7 +265,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
         issued = i + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA's memory goes away
-        for (int i = issued > AS ? issued - AS : 0; i < issued; ++i) {
+        for (int i = first; i < issued; i += 2) {
           const uint64_t t0 = global_timer_ns();
           while (!mbar_try_wait(act_full0 + 8 * (i % AS), (i / AS) & 1) && global_timer_ns() - t0 < limit) {
           }
@@ -290,9 +300,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
         }
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (elect_one()) {
+  } else if (warp == 1 || warp == T::kMmaWarpB) {
+    // ------------------------------------------------------- MMA issuers
+    constexpr int P = T::kMmaThreads;
+    constexpr int kOwnAccs = T::kAccs / P;  // accumulators per issuing thread
+    const int first = warp == 1 ? 0 : 1;
+    if (first < P && elect_one()) {
       constexpr uint32_t idesc = f16_instr_desc(128, BLOCK_T);
       // Descriptor of act stage 0; other stages and K steps add their byte
       // offset >> 4 to the start-address field (no carry: shared memory
@@ -301,8 +314,10 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
       // Software-pipelined: the waits for group i+1 sit between group i's
       // first six and last two MMAs, so the tensor core still has queued
       // work while this thread polls the barriers.
-      bool ready = ng > 0 && wait_phase(act_full0, 0, abort_flag, limit) && wait_phase(t_ready0, 0, abort_flag, limit);
-      for (int i = 0; ready && i < ng; ++i) {
+      bool ready = first < ng && wait_phase(act_full0 + 8 * (first % AS), (first / AS) & 1, abort_flag, limit) &&
+                   wait_phase(t_ready0 + 8 * (first % TS), (first / TS) & 1, abort_flag, limit);
+      int step = 0;  // this thread's MMA count
+      for (int i = first; ready && i < ng; i += P) {
         const int sa = i % AS, st = i % TS;
         tc_fence_after_sync();
         const uint64_t desc_s = desc0 + static_cast<uint64_t>((sa * T::kActStageBytes) >> 4);
@@ -310,15 +325,15 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
         bool next_ready = true;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          if (kk == 6 && i + 1 < ng) {
-            const int na = (i + 1) % AS, nt = (i + 1) % TS;
-            next_ready = wait_phase(act_full0 + 8 * na, ((i + 1) / AS) & 1, abort_flag, limit) &&
-                         wait_phase(t_ready0 + 8 * nt, ((i + 1) / TS) & 1, abort_flag, limit);
+          if (kk == 6 && i + P < ng) {
+            const int na = (i + P) % AS, nt = (i + P) % TS;
+            next_ready = wait_phase(act_full0 + 8 * na, ((i + P) / AS) & 1, abort_flag, limit) &&
+                         wait_phase(t_ready0 + 8 * nt, ((i + P) / TS) & 1, abort_flag, limit);
           }
           const uint64_t bdesc = desc_s + static_cast<uint64_t>(((kk >> 2) * T::kSliceBytes + (kk & 3) * 32) >> 4);
-          const int step = i * 8 + kk;
-          const uint32_t d = tmem + (step % T::kAccs) * BLOCK_T;
-          mma_f16_tmem_a(d, a_cols + kk * 8, bdesc, idesc, step >= T::kAccs ? 1u : 0u);
+          const int acc = (step % kOwnAccs) * P + first;
+          mma_f16_tmem_a(tmem + acc * BLOCK_T, a_cols + kk * 8, bdesc, idesc, step >= kOwnAccs ? 1u : 0u);
+          ++step;
         }
         mma_commit(act_empty0 + 8 * sa);
         mma_commit(t_free0 + 8 * st);
@@ -426,6 +441,8 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
     if (ok) ok = warp_wait(dfull, 0, abort_flag, limit);
     if (ok) tc_fence_after_sync();
     constexpr int kEpiCols = BLOCK_T / T::kEpiWarpsPerQuad;  // token columns per epilogue warp
+    // With two issuing threads and a single group, the second accumulator is unused.
+    const int used_accs = (T::kMmaThreads == 2 && ng < 2) ? 1 : T::kAccs;
     const bool epi = turn < T::kEpiWarpsPerQuad;
     const int c_begin = turn * kEpiCols;
     if (args.ksplit == 1) {
@@ -435,7 +452,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
 #pragma unroll 1
         for (int c = 0; c < kEpiCols; c += 8) {
           float acc[8];
-          sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, acc);
+          sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, used_accs, acc);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const __half h = __float2half_rn(acc[j] * T::kOutScale);
@@ -466,7 +483,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
 #pragma unroll 1
       for (int c = 0; c < kEpiCols; c += 8) {
         float acc[8];
-        sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, acc);
+        sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, used_accs, acc);
 #pragma unroll
         for (int j = 0; j < 8; ++j) part[(c_begin + c + j) * T::kRows + row] = acc[j];
       }
