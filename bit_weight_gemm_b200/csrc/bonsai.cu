@@ -283,14 +283,20 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   cfg.blockDim = dim3(T::kThreads);
   cfg.dynamicSmemBytes = T::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr;
+  // Programmatic dependent launch: the kernel's prologue may overlap the
+  // previous kernel in the stream; it waits for that kernel before touching
+  // global memory (griddepcontrol.wait), so stream order is preserved.
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
   if (ksplit > 1) {
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 1;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = ksplit;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = 1;
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = ksplit;
+    cfg.numAttrs = 2;
   }
   if (cudaLaunchKernelEx(&cfg, kernel, map_act, map_w, map_out, map_s, args) != cudaSuccess) return BONSAI_ERR_CUDA;
   return launch_status();

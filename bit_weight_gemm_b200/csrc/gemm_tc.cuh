@@ -25,6 +25,10 @@
 //                        accumulator in TMEM; tcgen05.commit releases the
 //                        act and TMEM stages.
 //
+// Launches use programmatic dependent launch: a CTA sets up its barriers and
+// tensor memory while the previous kernel in the stream finishes, and waits
+// for that kernel's completion before its first global-memory access.
+//
 // Epilogue, one CTA per tile (ksplit = 1): the converters read the
 // accumulator (tcgen05.ld), scale by 1 (binary) or 1/2 (ternary, exact),
 // round once to FP16 into a shared-memory tile, and one TMA store writes it.
@@ -215,6 +219,9 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
   const int ng = g_end - g_begin;
   const uint64_t limit = args.wait_limit_ns;
 
+  // The next launch in the stream may start its own prologue now; it waits
+  // (griddep_wait) for this grid to finish before touching global memory.
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < AS; ++s) {
       mbar_init(act_full0 + 8 * s, 1);
@@ -247,6 +254,10 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // Everything above touched only this CTA's own resources; global memory
+  // (activations, weights, scales, output) only after the preceding grid in
+  // the stream has completed.
+  griddep_wait();
 
   if (warp == 0 || warp == T::kActWarpB) {
     // ------------------------------------- activation producers (2, alternate groups)

@@ -114,6 +114,17 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
   return wait_phase_slow(bar, parity, abort_flag, limit_ns);
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// Blocks until every grid this one depends on has completed and its memory
+// writes are visible (a no-op when the launch has no such dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next grid in the stream be scheduled once every CTA of this grid
+// has issued this (or exited).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA --
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

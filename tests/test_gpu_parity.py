@@ -265,6 +265,46 @@ def test_gemm_matches_dequant_then_torch_matmul():
     assert bool(((got - ref).abs() <= bound).all())
 
 
+# ------------------------------------------------- back-to-back launches
+# Launches overlap their prologue with the previous kernel in the stream and
+# wait for it before touching global memory; these check both hazards.
+@pytest.mark.parametrize("M", [16, 4608])
+def test_chained_layers_read_after_write(oracle_mod, M):
+    K = 3072
+    d1 = workloads.make(mode="ternary", M=M, N=K, K=K, seed=71)
+    d2 = workloads.make(mode="binary", M=M, N=K, K=K, seed=72)
+    A = dev(d1["A"].view(np.int16), torch.float16)
+    p1, s1 = bw.pack(dev(d1["codes"]), "ternary"), dev(d1["scales"].view(np.int16), torch.float16)
+    p2, s2 = bw.pack(dev(d2["codes"]), "binary"), dev(d2["scales"].view(np.int16), torch.float16)
+    torch.cuda.synchronize()
+    h1 = bw.lowbit_gemm(A, p1, s1, "ternary")
+    h2 = bw.lowbit_gemm(h1, p2, s2, "binary")  # reads what the previous launch wrote
+    torch.cuda.synchronize()
+    h1_bits, h2_bits = to_u16(h1), to_u16(h2)
+    rng = np.random.default_rng(M)
+    ms, ns = rng.integers(0, M, 2000), rng.integers(0, K, 2000)
+    ref, _, absacc = oracle_mod.gemm_entries(h1_bits, oracle_mod.pack(d2["codes"], "binary"), d2["scales"], K,
+                                             "binary", ms, ns)
+    assert_gemm_close(oracle_mod, h2_bits[ms, ns], ref, absacc, f"chained layer 2, M={M}")
+
+
+def test_back_to_back_write_after_read(oracle_mod):
+    M = N = K = 3072
+    d = workloads.make(mode="ternary", M=M, N=N, K=K, seed=73)
+    A = dev(d["A"].view(np.int16), torch.float16)
+    packed, scales = bw.pack(dev(d["codes"]), "ternary"), dev(d["scales"].view(np.int16), torch.float16)
+    out = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    torch.cuda.synchronize()
+    bw.lowbit_gemm(A, packed, scales, "ternary", out=out)
+    bw.lowbit_gemm(out, packed, scales, "ternary", out=A)  # overwrites the input of the previous launch
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    ms, ns = rng.integers(0, M, 2000), rng.integers(0, N, 2000)
+    ref, _, absacc = oracle_mod.gemm_entries(d["A"], oracle_mod.pack(d["codes"], "ternary"), d["scales"], K,
+                                             "ternary", ms, ns)
+    assert_gemm_close(oracle_mod, to_u16(out)[ms, ns], ref, absacc, "first launch after a dependent overwrite")
+
+
 # ------------------------------------------------------------ edge cases
 def test_gemm_empty_shapes():
     A = torch.zeros((0, 128), dtype=torch.float16, device="cuda")
