@@ -259,75 +259,74 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
   // the stream has completed.
   griddep_wait();
 
+  // Producer and MMA loops run warp-uniformly: every lane of the warp takes
+  // the same path and waits, and one elected lane issues each TMA, arrive,
+  // MMA or commit (see the *_elected wrappers).
   if (warp == 0 || warp == T::kActWarpB) {
     // ------------------------------------- activation producers (2, alternate groups)
     const int first = warp == 0 ? 0 : 1;
-    if (elect_one()) {
-      int issued = 0;
-      for (int i = first; i < ng; i += 2) {
-        const int s = i % AS;
-        if (!wait_phase(act_empty0 + 8 * s, ((i / AS) & 1) ^ 1, abort_flag, limit)) break;
-        const uint32_t full = act_full0 + 8 * s;
-        mbar_arrive_expect_tx(full, T::kActStageBytes);
-        const uint32_t dst = smem_addr(smem + T::kActOff + s * T::kActStageBytes);
-        const int k = (g_begin + i) * kGroup;
-        tma_load_2d(dst, &tmap_act, full, k, m0);
-        tma_load_2d(dst + T::kSliceBytes, &tmap_act, full, k + 64, m0);
-        issued = i + 1;
-      }
-      if (*abort_flag) {  // let copies in flight land before the CTA's memory goes away
-        for (int i = first; i < issued; i += 2) {
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(act_full0 + 8 * (i % AS), (i / AS) & 1) && global_timer_ns() - t0 < limit) {
-          }
+    int issued = 0;
+    for (int i = first; i < ng; i += 2) {
+      const int s = i % AS;
+      if (!warp_wait(act_empty0 + 8 * s, ((i / AS) & 1) ^ 1, abort_flag, limit)) break;
+      const uint32_t full = act_full0 + 8 * s;
+      mbar_arrive_expect_tx_elected(full, T::kActStageBytes);
+      const uint32_t dst = smem_addr(smem + T::kActOff + s * T::kActStageBytes);
+      const int k = (g_begin + i) * kGroup;
+      tma_load_2d_elected(dst, &tmap_act, full, k, m0);
+      tma_load_2d_elected(dst + T::kSliceBytes, &tmap_act, full, k + 64, m0);
+      issued = i + 1;
+    }
+    if (*abort_flag) {  // let copies in flight land before the CTA's memory goes away
+      for (int i = first; i < issued; i += 2) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(act_full0 + 8 * (i % AS), (i / AS) & 1) && global_timer_ns() - t0 < limit) {
         }
       }
     }
   } else if (warp == 2) {
     // ------------------------------------------------ packed-word producer
-    if (elect_one()) {
-      if (args.scale_box > 0) {
-        // The tile's scales: 128 rows x scale_box groups from an 8-aligned
-        // group column (TMA needs 16-byte aligned starts).
-        mbar_arrive_expect_tx(s_full, static_cast<uint32_t>(args.scale_box) * T::kRows * 2);
-        tma_load_2d(smem_addr(smem + T::kScaleOff), &tmap_s, s_full, g_begin & ~7, n0);
-      }
-      int issued = 0;
-      const int nw = (ng + T::kWGroups - 1) / T::kWGroups;
-      for (int i = 0; i < nw; ++i) {
-        const int s = i % WS;
-        if (!wait_phase(w_empty0 + 8 * s, ((i / WS) & 1) ^ 1, abort_flag, limit)) break;
-        const uint32_t full = w_full0 + 8 * s;
-        mbar_arrive_expect_tx(full, T::kWStageBytes);
-        tma_load_2d(smem_addr(smem + T::kWOff + s * T::kWStageBytes), &tmap_w, full,
-                    (g_begin + i * T::kWGroups) * T::kWordsPerGroup, n0);
-        issued = i + 1;
-      }
-      if (*abort_flag) {
-        for (int i = issued > WS ? issued - WS : 0; i < issued; ++i) {
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(w_full0 + 8 * (i % WS), (i / WS) & 1) && global_timer_ns() - t0 < limit) {
-          }
+    if (args.scale_box > 0) {
+      // The tile's scales: 128 rows x scale_box groups from an 8-aligned
+      // group column (TMA needs 16-byte aligned starts).
+      mbar_arrive_expect_tx_elected(s_full, static_cast<uint32_t>(args.scale_box) * T::kRows * 2);
+      tma_load_2d_elected(smem_addr(smem + T::kScaleOff), &tmap_s, s_full, g_begin & ~7, n0);
+    }
+    int issued = 0;
+    const int nw = (ng + T::kWGroups - 1) / T::kWGroups;
+    for (int i = 0; i < nw; ++i) {
+      const int s = i % WS;
+      if (!warp_wait(w_empty0 + 8 * s, ((i / WS) & 1) ^ 1, abort_flag, limit)) break;
+      const uint32_t full = w_full0 + 8 * s;
+      mbar_arrive_expect_tx_elected(full, T::kWStageBytes);
+      tma_load_2d_elected(smem_addr(smem + T::kWOff + s * T::kWStageBytes), &tmap_w, full,
+                          (g_begin + i * T::kWGroups) * T::kWordsPerGroup, n0);
+      issued = i + 1;
+    }
+    if (*abort_flag) {
+      for (int i = issued > WS ? issued - WS : 0; i < issued; ++i) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(w_full0 + 8 * (i % WS), (i / WS) & 1) && global_timer_ns() - t0 < limit) {
         }
       }
     }
   } else if (warp == 1 || warp == T::kMmaWarpB) {
     // ------------------------------------------------------- MMA issuers
     constexpr int P = T::kMmaThreads;
-    constexpr int kOwnAccs = T::kAccs / P;  // accumulators per issuing thread
+    constexpr int kOwnAccs = T::kAccs / P;  // accumulators per issuing warp
     const int first = warp == 1 ? 0 : 1;
-    if (first < P && elect_one()) {
+    if (first < P) {
       constexpr uint32_t idesc = f16_instr_desc(128, BLOCK_T);
       // Descriptor of act stage 0; other stages and K steps add their byte
       // offset >> 4 to the start-address field (no carry: shared memory
       // addresses stay below 256 KB).
       const uint64_t desc0 = sw128_kmajor_desc(smem_addr(smem + T::kActOff));
-      // Software-pipelined: the waits for group i+1 sit between group i's
-      // first six and last two MMAs, so the tensor core still has queued
-      // work while this thread polls the barriers.
-      bool ready = first < ng && wait_phase(act_full0 + 8 * (first % AS), (first / AS) & 1, abort_flag, limit) &&
-                   wait_phase(t_ready0 + 8 * (first % TS), (first / TS) & 1, abort_flag, limit);
-      int step = 0;  // this thread's MMA count
+      // The waits for this warp's next group sit between the current group's
+      // sixth and seventh MMA, so the tensor core still has queued work while
+      // the warp polls the barriers.
+      bool ready = first < ng && warp_wait(act_full0 + 8 * (first % AS), (first / AS) & 1, abort_flag, limit) &&
+                   warp_wait(t_ready0 + 8 * (first % TS), (first / TS) & 1, abort_flag, limit);
+      int step = 0;  // this warp's MMA count
       for (int i = first; ready && i < ng; i += P) {
         const int sa = i % AS, st = i % TS;
         tc_fence_after_sync();
@@ -338,19 +337,19 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
         for (int kk = 0; kk < 8; ++kk) {
           if (kk == 6 && i + P < ng) {
             const int na = (i + P) % AS, nt = (i + P) % TS;
-            next_ready = wait_phase(act_full0 + 8 * na, ((i + P) / AS) & 1, abort_flag, limit) &&
-                         wait_phase(t_ready0 + 8 * nt, ((i + P) / TS) & 1, abort_flag, limit);
+            next_ready = warp_wait(act_full0 + 8 * na, ((i + P) / AS) & 1, abort_flag, limit) &&
+                         warp_wait(t_ready0 + 8 * nt, ((i + P) / TS) & 1, abort_flag, limit);
           }
           const uint64_t bdesc = desc_s + static_cast<uint64_t>(((kk >> 2) * T::kSliceBytes + (kk & 3) * 32) >> 4);
           const int acc = (step % kOwnAccs) * P + first;
-          mma_f16_tmem_a(tmem + acc * BLOCK_T, a_cols + kk * 8, bdesc, idesc, step >= kOwnAccs ? 1u : 0u);
+          mma_f16_tmem_a_elected(tmem + acc * BLOCK_T, a_cols + kk * 8, bdesc, idesc, step >= kOwnAccs ? 1u : 0u);
           ++step;
         }
-        mma_commit(act_empty0 + 8 * sa);
-        mma_commit(t_free0 + 8 * st);
+        mma_commit_elected(act_empty0 + 8 * sa);
+        mma_commit_elected(t_free0 + 8 * st);
         ready = next_ready;
       }
-      mma_commit(dfull);  // also on abort: lets this thread see its MMAs drain
+      mma_commit_elected(dfull);  // also on abort: lets this warp see its MMAs drain
       if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(dfull, 0) && global_timer_ns() - t0 < limit) {

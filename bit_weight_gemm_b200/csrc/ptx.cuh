@@ -40,6 +40,13 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// Warp-uniform issue.  The *_elected wrappers below are executed by a whole
+// converged warp; one lane, chosen by elect.sync inside the instruction
+// sequence (always the same lane for a full warp), issues the operation.  A
+// loop that stays warp-uniform keeps its descriptors and addresses in the
+// warp's uniform registers; the same loop run by one elected thread pays for
+// moving them on every tcgen05.mma (about three times the issue cost).
+
 // ------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -56,6 +63,17 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_elected(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred e;\n"
+      "  elect.sync _|e, 0xffffffff;\n"
+      "  @e mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;\n"
+      "}\n" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
@@ -137,6 +155,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_elected(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t x,
+                                                    int32_t y) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred e;\n"
+      "  elect.sync _|e, 0xffffffff;\n"
+      "  @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n"
+      "}\n" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
       : "memory");
 }
@@ -234,6 +264,30 @@ __device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem,
       "  tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
       "}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_f16_tmem_a_elected(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred p, e;\n"
+      "  setp.ne.b32 p, %4, 0;\n"
+      "  elect.sync _|e, 0xffffffff;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The elected lane (the one that issued the MMAs) commits.
+__device__ __forceinline__ void mma_commit_elected(uint32_t bar) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred e;\n"
+      "  elect.sync _|e, 0xffffffff;\n"
+      "  @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n"
+      "}\n" ::"r"(bar)
       : "memory");
 }
 
