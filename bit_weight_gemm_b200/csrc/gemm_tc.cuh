@@ -209,7 +209,10 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::kMiscOff + 4);
 
-  const int warp = threadIdx.x >> 5;
+  // Broadcast from lane 0 so that the compiler treats the warp index, and so
+  // every role branch below, as warp-uniform: the tcgen05 and TMA operands
+  // derived from it can then live in uniform registers.
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * T::kRows;
   const int m0 = blockIdx.y * BLOCK_T;
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);  // warp-uniform (see above)
   // Everything above touched only this CTA's own resources; global memory
   // (activations, weights, scales, output) only after the preceding grid in
   // the stream has completed.
