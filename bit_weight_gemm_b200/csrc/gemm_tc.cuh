@@ -324,25 +324,16 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
       // offset >> 4 to the start-address field (no carry: shared memory
       // addresses stay below 256 KB).
       const uint64_t desc0 = sw128_kmajor_desc(smem_addr(smem + T::kActOff));
-      // The waits for this warp's next group sit between the current group's
-      // sixth and seventh MMA, so the tensor core still has queued work while
-      // the warp polls the barriers.
-      bool ready = first < ng && warp_wait(act_full0 + 8 * (first % AS), (first / AS) & 1, abort_flag, limit) &&
-                   warp_wait(t_ready0 + 8 * (first % TS), (first / TS) & 1, abort_flag, limit);
       int step = 0;  // this warp's MMA count
-      for (int i = first; ready && i < ng; i += P) {
+      for (int i = first; i < ng; i += P) {
         const int sa = i % AS, st = i % TS;
+        if (!warp_wait(act_full0 + 8 * sa, (i / AS) & 1, abort_flag, limit)) break;
+        if (!warp_wait(t_ready0 + 8 * st, (i / TS) & 1, abort_flag, limit)) break;
         tc_fence_after_sync();
         const uint64_t desc_s = desc0 + static_cast<uint64_t>((sa * T::kActStageBytes) >> 4);
         const uint32_t a_cols = tmem + T::kACol0 + st * 64;
-        bool next_ready = true;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          if (kk == 6 && i + P < ng) {
-            const int na = (i + P) % AS, nt = (i + P) % TS;
-            next_ready = warp_wait(act_full0 + 8 * na, ((i + P) / AS) & 1, abort_flag, limit) &&
-                         warp_wait(t_ready0 + 8 * nt, ((i + P) / TS) & 1, abort_flag, limit);
-          }
           const uint64_t bdesc = desc_s + static_cast<uint64_t>(((kk >> 2) * T::kSliceBytes + (kk & 3) * 32) >> 4);
           const int acc = (step % kOwnAccs) * P + first;
           mma_f16_tmem_a_elected(tmem + acc * BLOCK_T, a_cols + kk * 8, bdesc, idesc, step >= kOwnAccs ? 1u : 0u);
@@ -350,7 +341,6 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
         }
         mma_commit_elected(act_empty0 + 8 * sa);
         mma_commit_elected(t_free0 + 8 * st);
-        ready = next_ready;
       }
       mma_commit_elected(dfull);  // also on abort: lets this warp see its MMAs drain
       if (*abort_flag) {
