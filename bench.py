@@ -155,6 +155,20 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- helpers
+def max_over_ranks(torch, seconds: float, dist=None, device="cuda") -> float:
+    """The slowest rank's time: every rank contributes its own device time."""
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_step: float, steps: int, world: int, seconds_max: float) -> float:
+    """Aggregate throughput: every rank ran `steps` steps of the same work
+    (weak scaling), in the slowest rank's time."""
+    return work_per_step * steps * world / seconds_max
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -327,12 +341,9 @@ def run_bonsai(args):
             sampler.start()
         secs = time_launches(torch, bw, p, sets, args.steps, args.warmup, dist)
         clocks = sampler.stop() if sampler else None
-        t = torch.tensor([secs], dtype=torch.float64, device="cuda")
-        if dist is not None:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        secs_max = float(t.item())
+        secs_max = max_over_ranks(torch, secs, dist)
         per_launch = secs_max / args.steps
-        value = flops(p) * args.steps * world / secs_max / 1e12
+        value = whole_job_rate(flops(p), args.steps, world, secs_max) / 1e12
         peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         achieved = flops(p) / per_launch / 1e12
         result.update(value=value, ms_per_step=per_launch * 1e3, clocks=clocks, achieved=achieved, peak=peak)
@@ -349,6 +360,7 @@ def run_bonsai(args):
     stack = None
     if not args.no_extras and not args.small_only:
         stack = [time_stack(torch, bw, m, "ternary", 20, 3) for m in (4608, 1024)]
+        stack.append(time_stack(torch, bw, 4608, "ternary", 20, 3, split_qkv=True))
 
     if dist is not None:
         dist.barrier()
@@ -412,11 +424,9 @@ def time_e2e(torch, bw, p, steps, warmup, dist):
     end.record(stream)
     torch.cuda.synchronize()
     secs = start.elapsed_time(end) / 1e3
-    t = torch.tensor([secs], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
     world = dist.get_world_size() if dist is not None else 1
-    return {"value": flops(p) * steps * world / float(t.item()) / 1e12, "unit": UNIT,
+    secs_max = max_over_ranks(torch, secs, dist)
+    return {"value": whole_job_rate(flops(p), steps, world, secs_max) / 1e12, "unit": UNIT,
             "h2d_bytes_per_step": 2 * p.M * p.K, "d2h_bytes_per_step": 2 * p.M * p.N, "steps": steps}
 
 
@@ -426,10 +436,7 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
     sets = make_sets(p, 64, torch, bw, distinct_weights=False)
     steps = max(args.steps, 200)
     secs = time_launches(torch, bw, p, sets, steps, max(args.warmup, 10), dist)
-    t = torch.tensor([secs], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    per_launch = float(t.item()) / steps
+    per_launch = max_over_ranks(torch, secs, dist) / steps
     nbytes = algorithmic_bytes(p)
     achieved = nbytes / per_launch / 1e9
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -443,11 +450,12 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
             "gpu_launches": steps}
 
 
-def time_stack(torch, bw, M, mode, steps, warmup, seed=2000):
-    """One denoise step of the 25-block MMDiT stack (80 launches = 100 linears,
-    Q|K|V stacked): every layer has its own weight buffers (cloned from one
-    seeded set per distinct shape), the step is captured as one CUDA graph."""
-    layers = workloads.mmdit_stack_layers()
+def time_stack(torch, bw, M, mode, steps, warmup, seed=2000, split_qkv=False):
+    """One denoise step of the 25-block MMDiT stack (80 launches = 100 linears
+    with Q|K|V stacked, or 100 launches with split_qkv): every layer has its
+    own weight buffers (cloned from one seeded set per distinct shape), the
+    step is captured as one CUDA graph."""
+    layers = workloads.mmdit_stack_layers(split_qkv=split_qkv)
     shapes = sorted({(n, k) for _, n, k in layers})
     base = {}
     for j, (n, k) in enumerate(shapes):

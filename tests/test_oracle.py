@@ -368,3 +368,13 @@ def test_page_sizes_are_consistent():
     assert 0.02 < frac < 0.08
     assert round(tb["full_precision"] / tb["binary"], 1) == g["transformer_reduction"]["binary"]
     assert round(tb["full_precision"] / tb["ternary"], 1) == g["transformer_reduction"]["ternary"]
+
+
+def test_stack_layer_lists():
+    """80 launches with Q|K|V stacked and 100 with them split cover the same
+    weights: 2,831,155,200 for a hidden-3072, 25-block MMDiT."""
+    fused = workloads.mmdit_stack_layers()
+    split = workloads.mmdit_stack_layers(split_qkv=True)
+    assert len(fused) == 80 and len(split) == 100
+    total = sum(n * k for _, n, k in fused)
+    assert total == sum(n * k for _, n, k in split) == 2_831_155_200

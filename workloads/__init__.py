@@ -54,16 +54,20 @@ CONFIGS = [
 ]
 
 
-def mmdit_stack_layers(hidden: int = 3072):
+def mmdit_stack_layers(hidden: int = 3072, split_qkv: bool = False):
     """(name, N, K) of the low-bit linears in one denoise step of a 25-block
     MMDiT: 5 double-stream blocks (two streams each with QKV, attention-out,
     MLP-up, MLP-down) and 20 single-stream blocks (fused QKV+MLP-up, fused
-    out).  Q|K|V are stacked, so 80 launches cover 100 linears."""
+    out).  With Q|K|V stacked, 80 launches cover the 100 linears; with
+    split_qkv the double-stream Q, K and V are separate launches (100)."""
     h = hidden
     layers = []
     for b in range(5):
         for stream in ("img", "txt"):
-            layers.append((f"double{b}.{stream}.qkv", 3 * h, h))
+            if split_qkv:
+                layers += [(f"double{b}.{stream}.{x}", h, h) for x in ("q", "k", "v")]
+            else:
+                layers.append((f"double{b}.{stream}.qkv", 3 * h, h))
             layers.append((f"double{b}.{stream}.out", h, h))
             layers.append((f"double{b}.{stream}.mlp_up", 3 * h, h))
             layers.append((f"double{b}.{stream}.mlp_down", h, 3 * h))
