@@ -176,7 +176,7 @@ def dist_setup(args):
     return world, rank, local
 
 
-def cpu_baseline(problem, budget_s: float = 12.0, rows: int = 64):
+def cpu_baseline(problem, budget_s: float = 15.0, rows: int = 512):
     """The oracle, as it stands, on a bounded sample of the workload: `rows`
     token rows against as many weight rows as fit the time budget."""
     import oracle
