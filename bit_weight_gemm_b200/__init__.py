@@ -32,7 +32,8 @@ SIGNATURES = {
     "bonsai_dequant": (ctypes.c_int, [_P, _P, _I64, _I64, ctypes.c_int, _P, _P]),
     "bonsai_lowbit_gemm": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P]),
     "bonsai_gemm_plan": (ctypes.c_int, [_I64, _I64, _I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
-                                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+                                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                                        ctypes.POINTER(ctypes.c_int)]),
     "bonsai_get_device_error": (ctypes.c_int, []),
     "bonsai_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bonsai_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint64]),
@@ -144,11 +145,12 @@ def lowbit_gemm(A: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, mod
 
 
 def gemm_plan(M: int, N: int, K: int, mode) -> dict:
-    """The launch bonsai_lowbit_gemm makes: tokens per tile, K split, CTAs."""
-    bt, ks, ctas = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    _check(lib().bonsai_gemm_plan(M, N, K, _mode(mode), ctypes.byref(bt), ctypes.byref(ks), ctypes.byref(ctas)),
-           "bonsai_gemm_plan")
-    return {"block_t": bt.value, "ksplit": ks.value, "ctas": ctas.value}
+    """The launch bonsai_lowbit_gemm makes: tokens per tile, K split, CTAs,
+    output tiles (fewer CTAs than tiles x split: the persistent form)."""
+    bt, ks, ctas, tiles = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().bonsai_gemm_plan(M, N, K, _mode(mode), ctypes.byref(bt), ctypes.byref(ks), ctypes.byref(ctas),
+                                  ctypes.byref(tiles)), "bonsai_gemm_plan")
+    return {"block_t": bt.value, "ksplit": ks.value, "ctas": ctas.value, "tiles": tiles.value}
 
 
 def get_device_error() -> int:

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "bonsai.h"
+#include "gemm_persistent.cuh"
 #include "gemm_tc.cuh"
 #include "pack_dequant.cuh"
 
@@ -302,6 +303,57 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   return launch_status();
 }
 
+// Persistent form (gemm_persistent.cuh): more 256-token tiles than SMs and
+// whole word stages per tile.
+template <int MODE>
+bool use_persistent(int M, int N, int K) {
+  using T = PersistTile<MODE>;
+  if (M <= 128 || K % (kGroup * T::kWGroups) != 0) return false;
+  const int64_t tiles = static_cast<int64_t>((N + T::kRows - 1) / T::kRows) * ((M + T::kBlockT - 1) / T::kBlockT);
+  return tiles > sm_count();
+}
+
+template <int MODE>
+int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
+                           uint16_t* out, cudaStream_t stream) {
+  using T = PersistTile<MODE>;
+  auto kernel = lowbit_gemm_persistent_kernel<MODE>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return BONSAI_ERR_CUDA;
+  CUtensorMap map_act, map_w;
+  const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
+  if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, T::kBlockT, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BONSAI_ERR_CUDA;
+  if (!make_map(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, words_per_row, N, 32, T::kRows,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return BONSAI_ERR_CUDA;
+  PersistArgs args;
+  args.scales = scales;
+  args.out = out;
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.tiles_n = (N + T::kRows - 1) / T::kRows;
+  args.tiles = args.tiles_n * ((M + T::kBlockT - 1) / T::kBlockT);
+  args.wait_limit_ns = kDefaultWaitLimitNs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(args.tiles < sm_count() ? args.tiles : sm_count());
+  cfg.blockDim = dim3(T::kThreads);
+  cfg.dynamicSmemBytes = T::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, map_act, map_w, args) != cudaSuccess) return BONSAI_ERR_CUDA;
+  return launch_status();
+}
+
 // More than 128 tokens: 256-token tiles, one CTA per SM.  (128-token tiles
 // at two CTAs per SM measured 15% slower on the M=4608 workload.)
 #ifndef BONSAI_LARGE_TILE
@@ -312,18 +364,22 @@ constexpr int kLargeTile = BONSAI_LARGE_TILE;
 constexpr int kLargeOcc = BONSAI_LARGE_OCC;
 
 struct Plan {
-  int block_t, ksplit, ctas;
+  int block_t, ksplit, ctas, tiles;
 };
 
 template <int MODE, int BLOCK_T, int OCC>
 Plan plan_for(int M, int N, int K) {
   const int tiles = ((N + 127) / 128) * ((M + BLOCK_T - 1) / BLOCK_T);
   const int ks = choose_ksplit<MODE, BLOCK_T, OCC>(tiles, K / kGroup);
-  return Plan{BLOCK_T, ks, tiles * ks};
+  return Plan{BLOCK_T, ks, tiles * ks, tiles};
 }
 
 template <int MODE>
 Plan plan_gemm(int M, int N, int K) {
+  if (use_persistent<MODE>(M, N, K)) {
+    const int tiles = ((N + 127) / 128) * ((M + 255) / 256);
+    return Plan{256, 1, sm_count(), tiles};
+  }
   if (M <= 16) return plan_for<MODE, 16, 1>(M, N, K);
   if (M <= 32) return plan_for<MODE, 32, 1>(M, N, K);
   if (M <= 64) return plan_for<MODE, 64, 1>(M, N, K);
@@ -334,6 +390,7 @@ Plan plan_gemm(int M, int N, int K) {
 template <int MODE>
 int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
                   uint16_t* out, cudaStream_t stream) {
+  if (use_persistent<MODE>(M, N, K)) return launch_gemm_persistent<MODE>(A, packed, scales, M, N, K, out, stream);
   if (M <= 16) return launch_gemm<MODE, 16, 1>(A, packed, scales, M, N, K, out, stream);
   if (M <= 32) return launch_gemm<MODE, 32, 1>(A, packed, scales, M, N, K, out, stream);
   if (M <= 64) return launch_gemm<MODE, 64, 1>(A, packed, scales, M, N, K, out, stream);
@@ -423,15 +480,16 @@ int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* sc
   return dispatch_gemm<BONSAI_TERNARY_INT2>(A, packed, scales, m, n, k, out, st);
 }
 
-int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas) {
+int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas, int* tiles) {
   if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
   int rc = check_shape(M, N, K);
   if (rc != BONSAI_OK) return rc;
-  if (!block_t || !ksplit || !ctas) return BONSAI_ERR_INVALID_ARG;
+  if (!block_t || !ksplit || !ctas || !tiles) return BONSAI_ERR_INVALID_ARG;
   if (M == 0 || N == 0 || K == 0) {
     *block_t = 0;
     *ksplit = 0;
     *ctas = 0;
+    *tiles = 0;
     return BONSAI_OK;
   }
   if ((rc = check_device()) != BONSAI_OK) return rc;
@@ -440,6 +498,7 @@ int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, in
   *block_t = p.block_t;
   *ksplit = p.ksplit;
   *ctas = p.ctas;
+  *tiles = p.tiles;
   return BONSAI_OK;
 }
 

@@ -97,9 +97,12 @@ int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* sc
 /* The launch bonsai_lowbit_gemm makes for this problem on the current
  * device: *block_t = tokens per tile (the MMA's N; each tile also covers 128
  * weight rows), *ksplit = CTAs that share one tile along K as a thread-block
- * cluster (1 = no split), *ctas = CTAs launched.  Host-side only (queries
+ * cluster (1 = no split), *ctas = CTAs launched, *tiles = output tiles.
+ * ctas < tiles x ksplit means the persistent form: one CTA per SM walks the
+ * tiles tau = blockIdx, blockIdx + ctas, ...  Host-side only (queries
  * occupancy, launches nothing).  Zero-sized problems report zeros. */
-int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas);
+int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas,
+                     int* tiles);
 
 /* Reads and clears the device-side error word of the current device: 0 if
  * no kernel reported a problem since the last call, else a bonsai_status

@@ -187,14 +187,41 @@ def test_gemm_full_size_sampled(oracle_mod, problem):
     assert np.isfinite(got.view(np.float16)).all()
 
 
-def test_plans_cover_both_epilogues():
-    big = bw.gemm_plan(4608, 9216, 3072, "ternary")
-    assert big["ksplit"] == 1 and big["block_t"] in (128, 256)
-    assert big["ctas"] == 72 * (4608 // big["block_t"])
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def test_plans_cover_every_form():
+    big = bw.gemm_plan(4608, 9216, 3072, "ternary")  # persistent: one CTA per SM walks 1296 tiles
+    assert big == {"block_t": 256, "ksplit": 1, "ctas": _sms(), "tiles": 72 * 18}
+    one_wave = bw.gemm_plan(1024, 3072, 3072, "binary")  # 96 tiles: one CTA (or cluster) each
+    assert one_wave["tiles"] == 24 * 4 and one_wave["ctas"] == one_wave["tiles"] * one_wave["ksplit"]
     for M, N, K in [(16, 3072, 9216), (16, 9216, 3072), (16, 256, 4096), (40, 384, 2048)]:
         p = bw.gemm_plan(M, N, K, "ternary")
-        assert 1 < p["ksplit"] <= 8 and p["ctas"] % p["ksplit"] == 0, (M, N, K, p)
-    assert bw.gemm_plan(0, 8, 128, "binary") == {"block_t": 0, "ksplit": 0, "ctas": 0}
+        assert 1 < p["ksplit"] <= 8 and p["ctas"] == p["tiles"] * p["ksplit"], (M, N, K, p)
+    assert bw.gemm_plan(0, 8, 128, "binary") == {"block_t": 0, "ksplit": 0, "ctas": 0, "tiles": 0}
+
+
+# Large M: more 256-token x 128-row tiles than SMs.  With K a multiple of 512
+# (ternary) or 1024 (binary) one persistent CTA per SM walks the tiles; else
+# each tile is its own CTA over several waves.  Ragged M and N; 186, 150 and
+# 237 tiles leave CTAs with one and with two tiles; N odd in the last case.
+LARGE_M_SHAPES = [
+    ("ternary", 1357, 3880, 512, True),
+    ("binary", 600, 6376, 1024, True),
+    ("ternary", 513, 9999, 1024, True),
+    ("ternary", 1357, 3880, 640, False),
+    ("binary", 600, 6376, 512, False),
+]
+
+
+@pytest.mark.parametrize("mode,M,N,K,persistent", LARGE_M_SHAPES)
+def test_gemm_large_m_full(oracle_mod, mode, M, N, K, persistent):
+    plan = bw.gemm_plan(M, N, K, mode)
+    assert plan["tiles"] > _sms() and plan["ksplit"] == 1
+    assert (plan["ctas"] < plan["tiles"]) == persistent, plan
+    got, ref, absacc = _gemm_case(oracle_mod, mode, M, N, K, seed=M + 3 * N + 7 * K)
+    assert_gemm_close(oracle_mod, got, ref, absacc, f"{mode} {M}x{N}x{K}")
 
 
 # ------------------------------------------------------------ invariants
