@@ -170,6 +170,26 @@ int sm_count() {
   return count[dev];
 }
 
+// Raises a kernel's dynamic shared-memory limit to what it uses, once per
+// device (the attribute is per device, and the occupancy queries below
+// depend on it).
+template <auto KERNEL>
+int smem_opt_in(int bytes) {
+  static std::mutex mu;
+  static bool done[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BONSAI_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return BONSAI_ERR_CUDA;
+    }
+    done[dev] = true;
+  }
+  return BONSAI_OK;
+}
+
 // Clusters of `ksplit` CTAs that can be resident at once (0 if unknown).
 template <int MODE, int BLOCK_T, int OCC>
 int resident_clusters(int ksplit) {
@@ -178,6 +198,7 @@ int resident_clusters(int ksplit) {
   static int cache[9] = {0};
   std::lock_guard<std::mutex> lock(mu);
   if (ksplit < 1 || ksplit > 8) return 0;
+  if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T, OCC>>(T::kSmemBytes) != BONSAI_OK) return 0;
   if (cache[ksplit] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, ksplit);
@@ -226,12 +247,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
                 cudaStream_t stream) {
   using T = GemmTile<MODE, BLOCK_T, OCC>;
   auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T, OCC>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return BONSAI_ERR_CUDA;
+  if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T, OCC>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
 
   CUtensorMap map_act, map_w, map_out;
   const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
@@ -318,12 +334,7 @@ int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t
                            uint16_t* out, cudaStream_t stream) {
   using T = PersistTile<MODE>;
   auto kernel = lowbit_gemm_persistent_kernel<MODE>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return BONSAI_ERR_CUDA;
+  if (smem_opt_in<lowbit_gemm_persistent_kernel<MODE>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
   CUtensorMap map_act, map_w;
   const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
   if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, T::kBlockT, CU_TENSOR_MAP_SWIZZLE_128B))

@@ -249,6 +249,14 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
     tma_prefetch_map(&tmap_out);
     if (args.scale_box > 0) tma_prefetch_map(&tmap_s);
   }
+  if (warp == 2 && lane == 0) {
+    // The CTA's packed words and scales into L2 while the preceding grid may
+    // still run (they are read-only here; the copies into shared memory
+    // follow griddep_wait).
+    const int nw = (ng + T::kWGroups - 1) / T::kWGroups;
+    for (int i = 0; i < nw; ++i) tma_prefetch_l2_2d(&tmap_w, (g_begin + i * T::kWGroups) * T::kWordsPerGroup, n0);
+    if (args.scale_box > 0) tma_prefetch_l2_2d(&tmap_s, g_begin & ~7, n0);
+  }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), T::kTmemCols);
     tmem_relinquish();

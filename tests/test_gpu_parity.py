@@ -202,6 +202,24 @@ def test_plans_cover_every_form():
     assert bw.gemm_plan(0, 8, 128, "binary") == {"block_t": 0, "ksplit": 0, "ctas": 0, "tiles": 0}
 
 
+def test_plan_in_a_fresh_process_matches_launch():
+    """The plan query before any launch in the process (occupancy of the
+    split-K clusters depends on the kernels' shared-memory opt-in) gives the
+    plan a launch uses."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import json, bit_weight_gemm_b200 as bw; "
+            "print(json.dumps([bw.gemm_plan(16, 3072, 9216, 'ternary'), bw.gemm_plan(40, 384, 2048, 'binary')]))")
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    fresh = json.loads(res.stdout.strip().splitlines()[-1])
+    assert fresh[0]["ksplit"] > 1 and fresh[1]["ksplit"] > 1, fresh
+    assert fresh == [bw.gemm_plan(16, 3072, 9216, "ternary"), bw.gemm_plan(40, 384, 2048, "binary")]
+
+
 # Large M: more 256-token x 128-row tiles than SMs.  With K a multiple of 512
 # (ternary) or 1024 (binary) one persistent CTA per SM walks the tiles; else
 # each tile is its own CTA over several waves.  Ragged M and N; 186, 150 and
