@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--sets", type=int, default=4, help="rotating input sets (their sum exceeds L2)")
     ap.add_argument("--no-extras", action="store_true", help="skip small-M, e2e, CPU baseline, clocks")
     ap.add_argument("--small-only", action="store_true", help="time only the M=16 workload (for profiling)")
+    ap.add_argument("--m-sweep", action="store_true",
+                    help="time the GEMM over M = 16..4608 on the stack's five layer shapes and print one JSON line")
     return ap.parse_args()
 
 
@@ -361,6 +363,7 @@ def run_bonsai(args):
     if not args.no_extras and not args.small_only:
         stack = [time_stack(torch, bw, m, "ternary", 20, 3) for m in (4608, 1024)]
         stack.append(time_stack(torch, bw, 4608, "ternary", 20, 3, split_qkv=True))
+        stack += [time_stack(torch, bw, None, "ternary", 20, 3, streams=st) for st in ((4096, 512), (1024, 512))]
 
     if dist is not None:
         dist.barrier()
@@ -450,28 +453,34 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
             "gpu_launches": steps}
 
 
-def time_stack(torch, bw, M, mode, steps, warmup, seed=2000, split_qkv=False):
+def time_stack(torch, bw, M, mode, steps, warmup, seed=2000, split_qkv=False, streams=None):
     """One denoise step of the 25-block MMDiT stack (80 launches = 100 linears
     with Q|K|V stacked, or 100 launches with split_qkv): every layer has its
     own weight buffers (cloned from one seeded set per distinct shape), the
-    step is captured as one CUDA graph."""
-    layers = workloads.mmdit_stack_layers(split_qkv=split_qkv)
-    shapes = sorted({(n, k) for _, n, k in layers})
+    step is captured as one CUDA graph.  With streams = (image tokens, text
+    tokens) the double-stream linears run on their own stream's rows and the
+    single-stream ones on the joint sequence; otherwise every layer has M rows."""
+    if streams is not None:
+        layers = workloads.mmdit_stream_layers(*streams)
+    else:
+        layers = [(name, M, n, k) for name, n, k in workloads.mmdit_stack_layers(split_qkv=split_qkv)]
+    shapes = sorted({(n, k) for _, _, n, k in layers})
     base = {}
     for j, (n, k) in enumerate(shapes):
         d = workloads.make(mode=mode, M=1, N=n, K=k, seed=seed + j)
         packed = bw.pack(torch.from_numpy(d["codes"]).cuda(), mode)
         scales = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
         base[(n, k)] = (packed, scales)
-    weights = [tuple(t.clone() for t in base[(n, k)]) for _, n, k in layers]
+    weights = [tuple(t.clone() for t in base[(n, k)]) for _, _, n, k in layers]
     rng = np.random.default_rng(seed)
-    acts = {k: torch.from_numpy(workloads.activations(rng, M, k).view(np.int16)).view(torch.float16).cuda()
-            for k in {k for _, _, k in layers}}
-    outs = {n: torch.empty((M, n), dtype=torch.float16, device="cuda") for n in {n for _, n, _ in layers}}
+    acts = {(m, k): torch.from_numpy(workloads.activations(rng, m, k).view(np.int16)).view(torch.float16).cuda()
+            for m, k in sorted({(m, k) for _, m, _, k in layers})}
+    outs = {(m, n): torch.empty((m, n), dtype=torch.float16, device="cuda")
+            for m, n in sorted({(m, n) for _, m, n, _ in layers})}
 
     def step():
-        for (name, n, k), (packed, scales) in zip(layers, weights):
-            bw.lowbit_gemm(acts[k], packed, scales, mode, out=outs[n])
+        for (name, m, n, k), (packed, scales) in zip(layers, weights):
+            bw.lowbit_gemm(acts[(m, k)], packed, scales, mode, out=outs[(m, n)])
 
     step()
     torch.cuda.synchronize()
@@ -489,16 +498,63 @@ def time_stack(torch, bw, M, mode, steps, warmup, seed=2000, split_qkv=False):
     end.record()
     torch.cuda.synchronize()
     ms = start.elapsed_time(end) / steps
-    total_flops = sum(2 * M * n * k for _, n, k in layers)
-    wbytes = sum(n * k // (8 if mode == "binary" else 4) + 2 * n * (k // 128) for _, n, k in layers)
+    total_flops = sum(2 * m * n * k for _, m, n, k in layers)
+    wbytes = sum(n * k // (8 if mode == "binary" else 4) + 2 * n * (k // 128) for _, _, n, k in layers)
     del graph
-    return {"M": M, "mode": mode, "launches": len(layers), "ms_per_denoise_step": ms,
+    rows = {"M": M} if streams is None else {"image_tokens": streams[0], "text_tokens": streams[1]}
+    return {**rows, "mode": mode, "launches": len(layers), "ms_per_denoise_step": ms,
             "tflops": total_flops / (ms * 1e-3) / 1e12, "weight_bytes": wbytes,
             "weight_gbs": wbytes / (ms * 1e-3) / 1e9}
 
 
+SWEEP_M = (16, 32, 64, 128, 192, 256, 384, 512, 768, 1024, 1536, 2048, 3072, 4096, 4608)
+SWEEP_SHAPES = ((3072, 3072), (9216, 3072), (3072, 9216), (18432, 3072), (3072, 12288))
+
+
+def run_m_sweep(args):
+    """TFLOP/s and weight-stream GB/s of single launches over the token
+    counts an MMDiT step meets (text stream 512, image 1024 / 4096, joint
+    1536 / 4608) and the small-batch end, on the stack's layer shapes.
+    Each point rotates over enough input sets to exceed L2 four times."""
+    import torch
+
+    torch.cuda.set_device(0)
+    import bit_weight_gemm_b200 as bw
+
+    mode = "ternary"
+    points = []
+    for j, (n, k) in enumerate(SWEEP_SHAPES):
+        d = workloads.make(mode=mode, M=1, N=n, K=k, seed=3000 + j)
+        packed = bw.pack(torch.from_numpy(d["codes"]).cuda(), mode)
+        scales = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+        rng = np.random.default_rng(3100 + j)
+        a_all = torch.from_numpy(workloads.activations(rng, max(SWEEP_M), k).view(np.int16)).view(torch.float16).cuda()
+        for m in SWEEP_M:
+            p = workloads.Problem(f"sweep M={m} N={n} K={k}", mode, m, n, k, 0)
+            per_set = algorithmic_bytes(p)
+            count = int(min(64, max(2, -(-4 * 126 * 2 ** 20 // per_set))))
+            sets = [(a_all[:m].clone(), packed.clone(), scales.clone(),
+                     torch.empty((m, n), dtype=torch.float16, device="cuda")) for _ in range(count)]
+            est = max(flops(p) / 1.4e15, per_set / 6.0e12) + 3e-6
+            steps = int(min(2000, max(4 * count, 0.03 / est)))
+            steps -= steps % count
+            secs = time_launches(torch, bw, p, sets, steps, 3)
+            t = secs / steps
+            wbytes = n * k // 4 + 2 * n * (k // 128)
+            points.append({"M": m, "N": n, "K": k, "us": t * 1e6, "tflops": flops(p) / t / 1e12,
+                           "gbs": per_set / t / 1e9, "weight_gbs": wbytes / t / 1e9,
+                           "plan": bw.gemm_plan(m, n, k, mode)})
+            del sets
+        del packed, scales, a_all
+    assert bw.get_device_error() == 0
+    print(json.dumps({"m_sweep": points, "mode": mode, "timing": "CUDA graph replay, CUDA events"}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.m_sweep:
+        return run_m_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_bonsai(args)

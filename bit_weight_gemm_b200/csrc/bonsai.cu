@@ -221,30 +221,9 @@ int resident_clusters(int ksplit) {
   return cache[ksplit] > 0 ? cache[ksplit] : 0;
 }
 
-// Split K over a cluster when the tiles alone leave SMs idle: pick the split
-// that minimises waves x groups per CTA.
 template <int MODE, int BLOCK_T, int OCC>
-int choose_ksplit(int tiles, int groups) {
-  const int sms = sm_count() * OCC;
-  if (tiles >= sms) return 1;
-  int best = 1;
-  double best_cost = 1e30;
-  for (int ks = 1; ks <= 8 && ks <= groups; ++ks) {
-    const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T, OCC>(ks);
-    if (per_wave <= 0) continue;
-    const int waves = (tiles + per_wave - 1) / per_wave;
-    const double cost = static_cast<double>(waves) * ((groups + ks - 1) / ks) + 0.25 * ks;  // small cost per split
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = ks;
-    }
-  }
-  return best;
-}
-
-template <int MODE, int BLOCK_T, int OCC>
-int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, uint16_t* out,
-                cudaStream_t stream) {
+int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, int ksplit,
+                uint16_t* out, cudaStream_t stream) {
   using T = GemmTile<MODE, BLOCK_T, OCC>;
   auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T, OCC>;
   if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T, OCC>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
@@ -266,8 +245,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   }
   const int groups = K / kGroup;
   const int tiles_n = (N + T::kRows - 1) / T::kRows, tiles_m = (M + BLOCK_T - 1) / BLOCK_T;
-  const int ksplit = choose_ksplit<MODE, BLOCK_T, OCC>(tiles_n * tiles_m, groups);
-  if (ksplit > groups) return BONSAI_ERR_SHAPE;
+  if (ksplit < 1 || ksplit > 8 || ksplit > groups) return BONSAI_ERR_SHAPE;
   // Scale tile by TMA: rows of the scale matrix must be 16-byte multiples
   // (groups % 8 == 0); the box covers a CTA's groups from an 8-aligned start.
   CUtensorMap map_s = map_act;  // placeholder when unused
@@ -365,48 +343,94 @@ int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t
   return launch_status();
 }
 
-// More than 128 tokens: 256-token tiles, one CTA per SM.  (128-token tiles
-// at two CTAs per SM measured 15% slower on the M=4608 workload.)
-#ifndef BONSAI_LARGE_TILE
-#define BONSAI_LARGE_TILE 256
-#define BONSAI_LARGE_OCC 1
-#endif
-constexpr int kLargeTile = BONSAI_LARGE_TILE;
-constexpr int kLargeOcc = BONSAI_LARGE_OCC;
-
-struct Plan {
-  int block_t, ksplit, ctas, tiles;
+// ------------------------------------------------------------- planning --
+// Launch costs in microseconds, measured on a B200 with an M sweep of single
+// launches (16..4608 tokens on the MMDiT layer shapes, clocks under the power
+// cap of a long run): per 128-wide K group of one CTA, per wave of one-tile
+// CTAs (start, accumulator read-out, store, exit), and per split-K cluster
+// reduction.  The persistent kernel pays about 1 us per tile boundary
+// instead of a wave's start and end.
+struct TileCost {
+  double group, wave, reduce;
 };
 
-template <int MODE, int BLOCK_T, int OCC>
-Plan plan_for(int M, int N, int K) {
+constexpr TileCost tile_cost(int block_t) {
+  return block_t <= 32    ? TileCost{0.31, 1.5, 1.0}
+         : block_t == 64  ? TileCost{0.31, 2.0, 1.5}
+         : block_t == 128 ? TileCost{0.50, 2.5, 2.0}
+                          : TileCost{0.75, 3.0, 4.0};
+}
+constexpr double kLaunchCost = 2.5;
+constexpr double kPersistentBoundary = 1.0;
+
+struct Plan {
+  int block_t = 0, ksplit = 0, ctas = 0, tiles = 0;
+  bool persistent = false;
+  double cost = 1e30;
+};
+
+// Every split of K (1..8, a cluster of that many CTAs per tile) for
+// BLOCK_T-token tiles: waves x (groups per CTA + per-wave costs).
+template <int MODE, int BLOCK_T>
+void consider(int M, int N, int K, Plan* best) {
+  const int groups = K / kGroup;
   const int tiles = ((N + 127) / 128) * ((M + BLOCK_T - 1) / BLOCK_T);
-  const int ks = choose_ksplit<MODE, BLOCK_T, OCC>(tiles, K / kGroup);
-  return Plan{BLOCK_T, ks, tiles * ks, tiles};
+  const TileCost c = tile_cost(BLOCK_T);
+  const int sms = sm_count();
+  for (int ks = 1; ks <= 8 && ks <= groups; ++ks) {
+    const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T, 1>(ks);
+    if (per_wave <= 0) continue;
+    const int waves = (tiles + per_wave - 1) / per_wave;
+    const bool persistent = BLOCK_T == 256 && ks == 1 && use_persistent<MODE>(M, N, K);
+    const double per_wave_cost = ((groups + ks - 1) / ks) * c.group + (persistent ? kPersistentBoundary : c.wave) +
+                                 (ks > 1 ? c.reduce : 0.0);
+    const double cost = kLaunchCost + waves * per_wave_cost;
+    if (cost < best->cost) {
+      best->block_t = BLOCK_T;
+      best->ksplit = ks;
+      best->tiles = tiles;
+      best->persistent = persistent;
+      best->ctas = persistent ? (tiles < sms ? tiles : sms) : tiles * ks;
+      best->cost = cost;
+    }
+  }
 }
 
+// Tokens per tile: the smallest MMA N that covers M up to 128; above that
+// 128- or 256-token tiles, whichever the cost model prefers (256 amortises
+// each converted weight over twice the tokens, 128 wastes fewer rows and
+// fills more SMs at mid M).
 template <int MODE>
 Plan plan_gemm(int M, int N, int K) {
-  if (use_persistent<MODE>(M, N, K)) {
-    const int tiles = ((N + 127) / 128) * ((M + 255) / 256);
-    return Plan{256, 1, sm_count(), tiles};
+  Plan best;
+  if (M <= 16) {
+    consider<MODE, 16>(M, N, K, &best);
+  } else if (M <= 32) {
+    consider<MODE, 32>(M, N, K, &best);
+  } else if (M <= 64) {
+    consider<MODE, 64>(M, N, K, &best);
+  } else if (M <= 128) {
+    consider<MODE, 128>(M, N, K, &best);
+  } else {
+    consider<MODE, 128>(M, N, K, &best);
+    consider<MODE, 256>(M, N, K, &best);
   }
-  if (M <= 16) return plan_for<MODE, 16, 1>(M, N, K);
-  if (M <= 32) return plan_for<MODE, 32, 1>(M, N, K);
-  if (M <= 64) return plan_for<MODE, 64, 1>(M, N, K);
-  if (M <= 128) return plan_for<MODE, 128, 1>(M, N, K);
-  return plan_for<MODE, kLargeTile, kLargeOcc>(M, N, K);
+  return best;
 }
 
 template <int MODE>
 int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
                   uint16_t* out, cudaStream_t stream) {
-  if (use_persistent<MODE>(M, N, K)) return launch_gemm_persistent<MODE>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 16) return launch_gemm<MODE, 16, 1>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 32) return launch_gemm<MODE, 32, 1>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 64) return launch_gemm<MODE, 64, 1>(A, packed, scales, M, N, K, out, stream);
-  if (M <= 128) return launch_gemm<MODE, 128, 1>(A, packed, scales, M, N, K, out, stream);
-  return launch_gemm<MODE, kLargeTile, kLargeOcc>(A, packed, scales, M, N, K, out, stream);
+  const Plan p = plan_gemm<MODE>(M, N, K);
+  if (p.persistent) return launch_gemm_persistent<MODE>(A, packed, scales, M, N, K, out, stream);
+  switch (p.block_t) {
+    case 16: return launch_gemm<MODE, 16, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 32: return launch_gemm<MODE, 32, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 64: return launch_gemm<MODE, 64, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 128: return launch_gemm<MODE, 128, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 256: return launch_gemm<MODE, 256, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    default: return BONSAI_ERR_CUDA;  // no plan: the occupancy queries failed
+  }
 }
 
 }  // namespace
@@ -506,6 +530,7 @@ int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, in
   if ((rc = check_device()) != BONSAI_OK) return rc;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   const Plan p = mode == BONSAI_BINARY ? plan_gemm<BONSAI_BINARY>(m, n, k) : plan_gemm<BONSAI_TERNARY_INT2>(m, n, k);
+  if (p.block_t == 0) return BONSAI_ERR_CUDA;
   *block_t = p.block_t;
   *ksplit = p.ksplit;
   *ctas = p.ctas;

@@ -220,13 +220,14 @@ def test_plan_in_a_fresh_process_matches_launch():
     assert fresh == [bw.gemm_plan(16, 3072, 9216, "ternary"), bw.gemm_plan(40, 384, 2048, "binary")]
 
 
-# Large M: more 256-token x 128-row tiles than SMs.  With K a multiple of 512
-# (ternary) or 1024 (binary) one persistent CTA per SM walks the tiles; else
-# each tile is its own CTA over several waves.  Ragged M and N; 186, 150 and
-# 237 tiles leave CTAs with one and with two tiles; N odd in the last case.
+# Large M: more tiles than SMs.  With K a multiple of 512 (ternary) or 1024
+# (binary) one persistent CTA per SM walks the 256-token tiles; else each
+# 128- or 256-token tile is its own CTA over several waves.  Ragged M and N;
+# 186, 150 and 237 tiles leave persistent CTAs with one and with two tiles;
+# N odd in the third case.
 LARGE_M_SHAPES = [
     ("ternary", 1357, 3880, 512, True),
-    ("binary", 600, 6376, 1024, True),
+    ("binary", 700, 6376, 1024, True),
     ("ternary", 513, 9999, 1024, True),
     ("ternary", 1357, 3880, 640, False),
     ("binary", 600, 6376, 512, False),

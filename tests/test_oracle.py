@@ -378,3 +378,20 @@ def test_stack_layer_lists():
     assert len(fused) == 80 and len(split) == 100
     total = sum(n * k for _, n, k in fused)
     assert total == sum(n * k for _, n, k in split) == 2_831_155_200
+
+
+def test_stream_layer_lists():
+    """With real per-stream token counts each double-stream block has its
+    image and text linears on their own rows and the single-stream blocks run
+    on the joint sequence; the weights are the same 2,831,155,200."""
+    layers = workloads.mmdit_stream_layers(4096, 512)
+    assert len(layers) == 80
+    assert sum(n * k for _, _, n, k in layers) == 2_831_155_200
+    rows = {}
+    for name, m, _, _ in layers:
+        kind = "single" if name.startswith("single") else ("img" if ".img." in name else "txt")
+        rows.setdefault(kind, set()).add(m)
+    assert rows == {"img": {4096}, "txt": {512}, "single": {4608}}
+    # 5 blocks x (4 image + 4 text linears) + 20 x 2 single-stream ones
+    assert sum(1 for name, *_ in layers if ".img." in name) == 20
+    assert sum(1 for name, *_ in layers if ".txt." in name) == 20

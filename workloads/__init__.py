@@ -77,6 +77,22 @@ def mmdit_stack_layers(hidden: int = 3072, split_qkv: bool = False):
     return layers
 
 
+def mmdit_stream_layers(img_tokens: int, txt_tokens: int, hidden: int = 3072):
+    """(name, M, N, K) of the low-bit linears in one denoise step with the
+    real per-stream token counts: the double-stream blocks run their image
+    and text streams as separate linears (separate weights) on img_tokens and
+    txt_tokens rows, the single-stream blocks on the joint sequence.  1024^2
+    images give 4096 image tokens, 512^2 give 1024; the text stream is 512."""
+    joint = img_tokens + txt_tokens
+    out = []
+    for name, n, k in mmdit_stack_layers(hidden):
+        if name.startswith("double"):
+            out.append((name, img_tokens if ".img." in name else txt_tokens, n, k))
+        else:
+            out.append((name, joint, n, k))
+    return out
+
+
 def _streams(seed: int):
     ss = np.random.SeedSequence(seed)
     return [np.random.Generator(np.random.PCG64(s)) for s in ss.spawn(3)]
