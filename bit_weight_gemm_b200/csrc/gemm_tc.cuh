@@ -48,6 +48,12 @@
 
 namespace bonsai {
 
+__host__ __device__ constexpr int largest_divisor_at_most(int n, int cap) {
+  int d = cap < n ? cap : n;
+  while (n % d != 0) --d;
+  return d;
+}
+
 __host__ __device__ constexpr int pow2_at_least(int x) {
   int p = 32;
   while (p < x) p *= 2;
@@ -78,10 +84,14 @@ struct GemmTile {
   static constexpr int kWStages = (OCC == 2 || BLOCK_T >= 256) ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   static constexpr int kScaleBytes = (OCC == 2 || BLOCK_T >= 256) ? 0 : 32768;
-  static constexpr int kConvWarps = OCC == 2 ? 8 : 16;  // 2 or 4 per TMEM lane quadrant
+  // Converter warps: 2 or 4 per TMEM lane quadrant.  (Five per quadrant on
+  // narrow tiles measured 2-5% slower: their tensor-memory stores, not the
+  // number of groups in conversion, set the pace.)
+  static constexpr int kConvWarps = OCC == 2 ? 8 : 16;
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
-  // Epilogue: the quadrant's warps split the token columns, 8 at least each.
-  static constexpr int kEpiWarpsPerQuad = BLOCK_T / 8 < kWarpsPerQuad ? BLOCK_T / 8 : kWarpsPerQuad;
+  // Epilogue: the quadrant's warps split the token columns, 8 at least each:
+  // the most warps (up to kWarpsPerQuad) that divide BLOCK_T / 8.
+  static constexpr int kEpiWarpsPerQuad = largest_divisor_at_most(BLOCK_T / 8, kWarpsPerQuad);
   // Two MMA-issuing threads (alternate groups, separate accumulators) and
   // two activation producers for tiles of up to 128 tokens, where one thread
   // issuing every MMA and polling every barrier is the serial limit.  A
@@ -100,7 +110,11 @@ struct GemmTile {
   // it completed, so the number of stages is the number of groups in flight
   // between the converters and the tensor core.
   static constexpr int kTmemCols = 512 / OCC;
-  static constexpr int kTStages = (kTmemCols - kACol0) / 64;
+  static constexpr int kTStagesFit = (kTmemCols - kACol0) / 64;
+  // With two MMA-issuing warps the stage count has the parity of
+  // kWarpsPerQuad (one stage is left unused otherwise); see the assertion below.
+  static constexpr int kTStages =
+      (kMmaThreads == 2 && (kTStagesFit - kWarpsPerQuad) % 2 != 0) ? kTStagesFit - 1 : kTStagesFit;
   static constexpr int kActOff = 0;
   static constexpr int kWOff = kActStages * kActStageBytes;
   static constexpr int kScaleOff = kWOff + kWStages * kWStageBytes;
@@ -117,10 +131,16 @@ struct GemmTile {
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(OCC == 1 || OCC == 2, "one or two CTAs per SM");
   static_assert(kACol0 + kTStages * 64 <= kTmemCols && kTStages >= 2, "TMEM budget");
-  // A converter warp takes every kWarpsPerQuad-th group, so it can wait on a
-  // TMEM stage at most one use ahead of the MMAs only if there are at least
-  // that many stages; with fewer, a parity wait could match an older phase.
+  // Parity waits on a TMEM stage are unambiguous only if the converter is at
+  // most one use ahead of the MMAs: when a converter waits for the MMAs of
+  // group i - TS (stage reuse), those of group i - 2TS must be done.  Its own
+  // previous wait (group i - kWarpsPerQuad) saw group i - kWarpsPerQuad - TS
+  // done, which covers i - 2TS if kWarpsPerQuad <= TS and, with two MMA warps
+  // taking alternate groups, if both groups were issued by the same warp
+  // (whose commit covers all its earlier MMAs): TS - kWarpsPerQuad even.
   static_assert(kWarpsPerQuad <= kTStages, "converter warps per quadrant <= TMEM stages");
+  static_assert(kWGroups % kWarpsPerQuad == 0, "every converter warp reads every full word stage");
+  static_assert(kMmaThreads == 1 || (kTStages - kWarpsPerQuad) % 2 == 0, "same MMA warp for groups i-q-TS, i-2TS");
   static_assert(kSmemBytes <= (OCC == 1 ? 227 * 1024 : 113 * 1024), "shared memory per CTA");
   static_assert(kActStages >= 2, "activation ring depth");
   static_assert(BLOCK_T * kRows * 2 <= kActStages * kActStageBytes, "output tile fits the act ring");
@@ -440,7 +460,10 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
         words[7] = q1.w;
       }
       __syncwarp();
-      // Release the word stage after this warp's last group in it.
+      // Release the word stage after this warp's last group in it.  Every
+      // converter warp has a group in every full stage (kWGroups is a multiple
+      // of kWarpsPerQuad); only the CTA's last stage, which is never refilled,
+      // may lack some warps' arrivals.
       const int stage_end = (wj + 1) * T::kWGroups < ng ? (wj + 1) * T::kWGroups : ng;
       if (lane == 0 && i + kStep >= stage_end) mbar_arrive(w_empty0 + 8 * sw);
       convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);

@@ -311,6 +311,30 @@ def test_gemm_matches_dequant_then_torch_matmul():
     assert bool(((got - ref).abs() <= bound).all())
 
 
+# Narrow tiles with many groups per CTA: converters run up to one TMEM stage
+# use ahead of the MMAs, so a wrong stage count would let a parity wait match
+# an old phase (a timeout, or a stage overwritten while still read).  Many
+# back-to-back launches give the race its chances.
+@pytest.mark.parametrize("mode,M,N,K", [("ternary", 16, 3072, 12288), ("ternary", 32, 3072, 12288),
+                                        ("ternary", 64, 3072, 12288), ("ternary", 64, 9216, 3072),
+                                        ("binary", 64, 3072, 12288), ("ternary", 128, 3072, 12288)])
+def test_narrow_tiles_repeated_launches(oracle_mod, mode, M, N, K):
+    d = workloads.make(mode=mode, M=M, N=N, K=K, seed=M + N + K)
+    ref_packed, packed, A, scales = gpu_inputs(d, oracle_mod)
+    first = bw.lowbit_gemm(A, packed, scales, mode)
+    out = torch.empty_like(first)
+    torch.cuda.synchronize()
+    for _ in range(150):
+        bw.lowbit_gemm(A, packed, scales, mode, out=out)
+    torch.cuda.synchronize()
+    assert bw.get_device_error() == 0
+    assert torch.equal(out, first)
+    rng = np.random.default_rng(K)
+    ms, ns = rng.integers(0, M, 600), rng.integers(0, N, 600)
+    ref, _, absacc = oracle_mod.gemm_entries(d["A"], ref_packed, d["scales"], K, mode, ms, ns)
+    assert_gemm_close(oracle_mod, to_u16(first)[ms, ns], ref, absacc, f"{mode} {M}x{N}x{K}")
+
+
 # ------------------------------------------------- back-to-back launches
 # Launches overlap their prologue with the previous kernel in the stream and
 # wait for it before touching global memory; these check both hazards.
