@@ -31,6 +31,7 @@ SIGNATURES = {
     "bonsai_pack": (ctypes.c_int, [_P, _I64, _I64, ctypes.c_int, _P, _P]),
     "bonsai_dequant": (ctypes.c_int, [_P, _P, _I64, _I64, ctypes.c_int, _P, _P]),
     "bonsai_lowbit_gemm": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P]),
+    "bonsai_lowbit_gemm_host": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P]),
     "bonsai_gemm_plan": (ctypes.c_int, [_I64, _I64, _I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
                                         ctypes.POINTER(ctypes.c_int)]),
@@ -142,6 +143,43 @@ def lowbit_gemm(A: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, mod
                                     _dev(scales, "scales", torch.float16), M, N, K, m,
                                     _dev(out, "out", torch.float16), _stream()), "bonsai_lowbit_gemm")
     return out
+
+
+def _host(t: torch.Tensor, name: str) -> ctypes.c_void_p:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != torch.float16:
+        raise ValueError(f"{name} must be torch.float16, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def lowbit_gemm_host(A_host: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, mode,
+                     out_host: torch.Tensor | None = None, A_dev: torch.Tensor | None = None,
+                     out_dev: torch.Tensor | None = None) -> torch.Tensor:
+    """The GEMM with A and out in (pinned) host memory: chunked copies in,
+    GEMMs and copies out overlap on the library's streams; ordered on the
+    current stream and not synchronised.  A_dev / out_dev are the device work
+    buffers ([M,K] and [M,N] FP16), allocated here when not given."""
+    M, K = A_host.shape
+    N = packed.shape[0]
+    m = _mode(mode)
+    dev = packed.device
+    if out_host is None:
+        out_host = torch.empty((M, N), dtype=torch.float16, pin_memory=True)
+    if A_dev is None:
+        A_dev = torch.empty((M, K), dtype=torch.float16, device=dev)
+    if out_dev is None:
+        out_dev = torch.empty((M, N), dtype=torch.float16, device=dev)
+    if A_dev.numel() < M * K or out_dev.numel() < M * N or out_host.numel() < M * N:
+        raise ValueError("work or output buffer too small")
+    _check(lib().bonsai_lowbit_gemm_host(_host(A_host, "A_host"), _dev(packed, "packed"),
+                                         _dev(scales, "scales", torch.float16), M, N, K, m,
+                                         _host(out_host, "out_host"), _dev(A_dev, "A_dev", torch.float16),
+                                         _dev(out_dev, "out_dev", torch.float16), _stream()),
+           "bonsai_lowbit_gemm_host")
+    return out_host
 
 
 def gemm_plan(M: int, N: int, K: int, mode) -> dict:

@@ -433,6 +433,93 @@ int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales,
   }
 }
 
+// ------------------------------------------------ host-buffer pipeline --
+// Three streams per device (copies in, GEMMs, copies out) and the events that
+// chain a call's chunks, created on first use and kept for the process.
+constexpr int kMaxChunks = 16;
+
+struct HostPipeline {
+  bool ready = false;
+  cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t copied[kMaxChunks] = {}, computed[kMaxChunks] = {};
+};
+
+std::mutex g_pipe_mu;
+HostPipeline g_pipes[64];
+
+int pipeline_for_device(HostPipeline** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BONSAI_ERR_CUDA;
+  HostPipeline& p = g_pipes[dev];
+  if (!p.ready) {
+    const unsigned ev = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.comp, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&p.start, ev) == cudaSuccess &&
+              cudaEventCreateWithFlags(&p.done, ev) == cudaSuccess;
+    for (int c = 0; ok && c < kMaxChunks; ++c)
+      ok = cudaEventCreateWithFlags(&p.copied[c], ev) == cudaSuccess &&
+           cudaEventCreateWithFlags(&p.computed[c], ev) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return BONSAI_ERR_CUDA;  // partial objects are kept and retried next time
+    }
+    p.ready = true;
+  }
+  *out = &p;
+  return BONSAI_OK;
+}
+
+// Rows per chunk: a multiple of 256 (whole 256-token tiles), about a quarter
+// of M so that copies in, GEMMs and copies out of neighbouring chunks overlap,
+// and at most kMaxChunks chunks.
+int64_t chunk_rows(int64_t M) {
+  const int64_t quarter = (M + 3) / 4;
+  const int64_t cap = (M + kMaxChunks - 1) / kMaxChunks;
+  int64_t rows = quarter > cap ? quarter : cap;
+  rows = (rows + 255) / 256 * 256;
+  return rows < 256 ? 256 : rows;
+}
+
+template <int MODE>
+int gemm_host_pipelined(const uint16_t* A_host, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
+                        int64_t K, uint16_t* out_host, uint16_t* A_dev, uint16_t* out_dev, cudaStream_t user) {
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipeline* p = nullptr;
+  int rc = pipeline_for_device(&p);
+  if (rc != BONSAI_OK) return rc;
+  const int64_t rows = chunk_rows(M);
+  const int chunks = static_cast<int>((M + rows - 1) / rows);
+  // Fork: all three streams start after the work already on the caller's stream.
+  if (cudaEventRecord(p->start, user) != cudaSuccess || cudaStreamWaitEvent(p->in, p->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(p->comp, p->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(p->out, p->start, 0) != cudaSuccess)
+    return BONSAI_ERR_CUDA;
+  for (int c = 0; c < chunks; ++c) {
+    const int64_t r0 = c * rows, m = (M - r0) < rows ? (M - r0) : rows;
+    const size_t a_off = static_cast<size_t>(r0) * K, o_off = static_cast<size_t>(r0) * N;
+    if (cudaMemcpyAsync(A_dev + a_off, A_host + a_off, static_cast<size_t>(m) * K * 2, cudaMemcpyHostToDevice,
+                        p->in) != cudaSuccess ||
+        cudaEventRecord(p->copied[c], p->in) != cudaSuccess || cudaStreamWaitEvent(p->comp, p->copied[c], 0) != cudaSuccess)
+      return BONSAI_ERR_CUDA;
+    rc = dispatch_gemm<MODE>(A_dev + a_off, packed, scales, static_cast<int>(m), static_cast<int>(N),
+                             static_cast<int>(K), out_dev + o_off, p->comp);
+    if (rc != BONSAI_OK) return rc;
+    if (cudaEventRecord(p->computed[c], p->comp) != cudaSuccess ||
+        cudaStreamWaitEvent(p->out, p->computed[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(out_host + o_off, out_dev + o_off, static_cast<size_t>(m) * N * 2, cudaMemcpyDeviceToHost,
+                        p->out) != cudaSuccess)
+      return BONSAI_ERR_CUDA;
+  }
+  // Join: the caller's stream continues after the last copy out (which
+  // follows every chunk's GEMM and copy in).
+  if (cudaEventRecord(p->done, p->out) != cudaSuccess || cudaStreamWaitEvent(user, p->done, 0) != cudaSuccess)
+    return BONSAI_ERR_CUDA;
+  return BONSAI_OK;
+}
+
 }  // namespace
 }  // namespace bonsai
 
@@ -513,6 +600,28 @@ int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* sc
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   if (mode == BONSAI_BINARY) return dispatch_gemm<BONSAI_BINARY>(A, packed, scales, m, n, k, out, st);
   return dispatch_gemm<BONSAI_TERNARY_INT2>(A, packed, scales, m, n, k, out, st);
+}
+
+int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
+                            int64_t K, int mode, uint16_t* out_host, uint16_t* A_dev, uint16_t* out_dev, void* stream) {
+  if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
+  int rc = check_shape(M, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (M == 0 || N == 0) return BONSAI_OK;
+  if (!A_host || !out_host || !A_dev || !out_dev || (K > 0 && (!packed || !scales))) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(A_dev) || !aligned16(out_dev) || (K > 0 && (!aligned16(packed) || !aligned16(scales))))
+    return BONSAI_ERR_ALIGN;
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 0) {  // empty sum: zeros, written through the device buffer
+    if (cudaMemsetAsync(out_dev, 0, static_cast<size_t>(M) * N * 2, st) != cudaSuccess ||
+        cudaMemcpyAsync(out_host, out_dev, static_cast<size_t>(M) * N * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return BONSAI_ERR_CUDA;
+    return BONSAI_OK;
+  }
+  if (mode == BONSAI_BINARY)
+    return gemm_host_pipelined<BONSAI_BINARY>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
+  return gemm_host_pipelined<BONSAI_TERNARY_INT2>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
 }
 
 int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas, int* tiles) {

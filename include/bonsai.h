@@ -94,6 +94,26 @@ int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_
 int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int64_t M,
                        int64_t N, int64_t K, int mode, uint16_t* out, void* stream);
 
+/* The same GEMM with the activations and the output in host memory (the
+ * pages' layer applied to a batch that lives on the host; no counterpart of
+ * its own on the pages).  A_host: FP16 [M,K]; out_host: FP16 [M,N]; both
+ * should be page-locked (cudaHostAlloc / pinned) for the copies to overlap.
+ * packed/scales: device memory as for bonsai_lowbit_gemm.  A_dev and
+ * out_dev: caller-owned device work buffers of at least M*K and M*N FP16
+ * values, 16-byte aligned (the library allocates nothing).
+ * The rows are split into chunks of a multiple of 256; chunk c's
+ * host->device copy, GEMM and device->host copy run on three library-owned
+ * streams, so that the copies in both directions overlap the GEMMs of other
+ * chunks.  The work is ordered after everything already enqueued on `stream`
+ * and everything enqueued on `stream` afterwards is ordered after it; the
+ * call returns without synchronising.  Host buffers must stay valid and
+ * unmodified (A_host) / unread (out_host) until `stream` reaches that point.
+ * Errors: as bonsai_lowbit_gemm, plus BONSAI_ERR_INVALID_ARG for null
+ * pointers. */
+int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const uint16_t* scales, int64_t M,
+                            int64_t N, int64_t K, int mode, uint16_t* out_host, uint16_t* A_dev,
+                            uint16_t* out_dev, void* stream);
+
 /* The launch bonsai_lowbit_gemm makes for this problem on the current
  * device: *block_t = tokens per tile (the MMA's N; each tile also covers 128
  * weight rows), *ksplit = CTAs that share one tile along K as a thread-block

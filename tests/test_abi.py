@@ -29,7 +29,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for required in ["bonsai_pack", "bonsai_dequant", "bonsai_lowbit_gemm", "bonsai_get_device_error",
+    for required in ["bonsai_pack", "bonsai_dequant", "bonsai_lowbit_gemm", "bonsai_lowbit_gemm_host",
+                     "bonsai_get_device_error",
                      "bonsai_status_string", "bonsai_packed_bytes", "bonsai_scale_bytes"]:
         assert required in names
 
@@ -81,6 +82,14 @@ def test_argument_errors_before_any_device_work(lib):
     assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 128, 2, P, P) == 1
     assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 128, 2, 8, P) == 3
     assert lib.bonsai_lowbit_gemm(P, P, P, 1 << 31, 4, 128, 2, 16, P) == 2
+    # host-buffer form: A_host, packed, scales, M, N, K, mode, out_host, A_dev, out_dev, stream
+    H = 16
+    assert lib.bonsai_lowbit_gemm_host(H, H, H, 4, 4, 128, 0, H, H, H, P) == 1  # mode
+    assert lib.bonsai_lowbit_gemm_host(H, H, H, 4, 4, 129, 2, H, H, H, P) == 2  # K % 128
+    assert lib.bonsai_lowbit_gemm_host(P, P, P, 0, 4, 128, 2, P, P, P, P) == 0  # empty: no-op
+    assert lib.bonsai_lowbit_gemm_host(P, H, H, 4, 4, 128, 2, H, H, H, P) == 1  # null host input
+    assert lib.bonsai_lowbit_gemm_host(H, H, H, 4, 4, 128, 2, H, P, H, P) == 1  # null work buffer
+    assert lib.bonsai_lowbit_gemm_host(H, H, H, 4, 4, 128, 2, H, 8, H, P) == 3  # misaligned work buffer
 
 
 def test_status_strings(lib):

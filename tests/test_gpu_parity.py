@@ -335,6 +335,53 @@ def test_narrow_tiles_repeated_launches(oracle_mod, mode, M, N, K):
     assert_gemm_close(oracle_mod, to_u16(first)[ms, ns], ref, absacc, f"{mode} {M}x{N}x{K}")
 
 
+# Host buffers in and out: chunked copies and GEMMs on the library's streams,
+# ordered on the caller's stream.  Ragged M over several chunks, compared in
+# full; the headline workload at sampled positions; back-to-back calls that
+# reuse the same work buffers.
+@pytest.mark.parametrize("mode,M,N,K", [("ternary", 1357, 3880, 512), ("binary", 16, 3072, 1024),
+                                        ("ternary", 300, 256, 384)])
+def test_gemm_host_buffers_full(oracle_mod, mode, M, N, K):
+    d = workloads.make(mode=mode, M=M, N=N, K=K, seed=7 * M + N + K)
+    ref_packed = oracle_mod.pack(d["codes"], mode)
+    packed = bw.pack(dev(d["codes"]), mode)
+    scales = dev(d["scales"].view(np.int16), torch.float16)
+    A_host = torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).pin_memory()
+    out_host = bw.lowbit_gemm_host(A_host, packed, scales, mode)
+    torch.cuda.synchronize()
+    ref, _, absacc = oracle_mod.gemm(d["A"], ref_packed, d["scales"], K, mode)
+    assert_gemm_close(oracle_mod, out_host.view(torch.int16).numpy().view(np.uint16), ref, absacc,
+                      f"host buffers {mode} {M}x{N}x{K}")
+
+
+def test_gemm_host_buffers_headline_and_reuse(oracle_mod):
+    p = workloads.TERNARY_MLP_UP_4608
+    d = workloads.make(p)
+    ref_packed = oracle_mod.pack(d["codes"], p.mode)
+    packed = bw.pack(dev(d["codes"]), p.mode)
+    scales = dev(d["scales"].view(np.int16), torch.float16)
+    A_host = torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).pin_memory()
+    A2_host = (A_host.float() * -2.0).half().pin_memory()  # exact: the output negates and doubles
+    A_dev = torch.empty((p.M, p.K), dtype=torch.float16, device="cuda")
+    out_dev = torch.empty((p.M, p.N), dtype=torch.float16, device="cuda")
+    out1 = torch.empty((p.M, p.N), dtype=torch.float16).pin_memory()
+    out2 = torch.empty((p.M, p.N), dtype=torch.float16).pin_memory()
+    bw.lowbit_gemm_host(A_host, packed, scales, p.mode, out_host=out1, A_dev=A_dev, out_dev=out_dev)
+    bw.lowbit_gemm_host(A2_host, packed, scales, p.mode, out_host=out2, A_dev=A_dev, out_dev=out_dev)
+    torch.cuda.synchronize()
+    assert bw.get_device_error() == 0
+    got = out1.view(torch.int16).numpy().view(np.uint16)
+    ms, ns = _sample_positions(p.M, p.N, 256, 3000, p.seed)
+    ref, _, absacc = oracle_mod.gemm_entries(d["A"], ref_packed, d["scales"], p.K, p.mode, ms, ns)
+    assert_gemm_close(oracle_mod, got[ms, ns], ref, absacc, "host buffers, headline workload")
+    # The second call (same plans, same summation order) against the first,
+    # exactly, through the scaling invariant: -2 scales the FP32 sum exactly
+    # and commutes with rounding wherever the result is a normal FP16 number.
+    normal = out1.float().abs() >= 2.0 ** -13
+    assert bool(normal.float().mean() > 0.99)
+    assert torch.equal(out2[normal], (out1.float() * -2.0).half()[normal])
+
+
 # ------------------------------------------------- back-to-back launches
 # Launches overlap their prologue with the previous kernel in the stream and
 # wait for it before touching global memory; these check both hazards.
