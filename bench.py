@@ -364,6 +364,10 @@ def run_bonsai(args):
         stack = [time_stack(torch, bw, m, "ternary", 20, 3) for m in (4608, 1024)]
         stack.append(time_stack(torch, bw, 4608, "ternary", 20, 3, split_qkv=True))
         stack += [time_stack(torch, bw, None, "ternary", 20, 3, streams=st) for st in ((4096, 512), (1024, 512))]
+        stack += [time_stack(torch, bw, m, "binary", 20, 3) for m in (4608, 1024)]
+    cublas = None
+    if not args.no_extras and not args.small_only:
+        cublas = cublas_fp16_same_run(torch)
 
     if dist is not None:
         dist.barrier()
@@ -382,7 +386,8 @@ def run_bonsai(args):
                                  f"total > 126 MB L2"},
                 "roofline": {"bound": "tensor", "achieved": result["achieved"], "peak": result["peak"],
                              "unit": "TFLOP/s", "frac": result["achieved"] / result["peak"],
-                             "traffic": traffic, "peak_source": f"{peaks_kind} bf16 dense (fp16 same nominal rate)"},
+                             "traffic": traffic, "peak_source": f"{peaks_kind} bf16 dense (fp16 same nominal rate)",
+                             "cublas_fp16_same_run": cublas},
                 "gpu_launches": args.steps,
                 "timing": "CUDA graph replay of the launches, CUDA events on the replay stream",
                 "clocks": result["clocks"],
@@ -452,6 +457,39 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
                          "frac": achieved / peak, "traffic": ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}"),
                          "algorithmic_bytes_per_launch": nbytes, "peak_source": f"{peaks_kind} hbm copy"},
             "gpu_launches": steps}
+
+
+def cublas_fp16_same_run(torch, n=8192, seconds=0.4):
+    """Dense FP16 torch.matmul (cuBLAS) n^3 on this GPU in this run, for
+    context beside the measured peaks: best of 10 single launches, and the
+    mean over about `seconds` of back-to-back launches (the length of the
+    headline's timed region, so under the same power cap)."""
+    a = torch.randn((n, n), device="cuda", dtype=torch.float16)
+    b = torch.randn((n, n), device="cuda", dtype=torch.float16)
+    c = torch.empty((n, n), device="cuda", dtype=torch.float16)
+    flop = 2.0 * n ** 3
+    for _ in range(3):
+        torch.matmul(a, b, out=c)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.matmul(a, b, out=c)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1) / 1e3)
+    reps = max(10, int(seconds / best))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        torch.matmul(a, b, out=c)
+    e1.record()
+    torch.cuda.synchronize()
+    loop = e0.elapsed_time(e1) / 1e3 / reps
+    del a, b, c
+    return {"burst_tflops": flop / best / 1e12, "loop_tflops": flop / loop / 1e12, "loop_launches": reps,
+            "shape": f"{n}^3 fp16"}
 
 
 def time_stack(torch, bw, M, mode, steps, warmup, seed=2000, split_qkv=False, streams=None):

@@ -23,6 +23,7 @@ import numpy as np
 
 BINARY = 1
 TERNARY = 2
+TERNARY_B3 = 3  # five trits per byte, this project's denser format (see bonsai_oracle.c)
 GROUP = 128
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -101,6 +102,8 @@ def _mode(mode) -> int:
         return BINARY
     if mode in (TERNARY, "ternary"):
         return TERNARY
+    if mode in (TERNARY_B3, "ternary_b3"):
+        return TERNARY_B3
     raise ValueError(f"unknown mode {mode!r}")
 
 
@@ -131,11 +134,15 @@ def packed_bytes(N: int, K: int, mode) -> int:
 
 
 def words_per_row(K: int, mode) -> int:
-    return K // (32 if _mode(mode) == BINARY else 16)
+    m = _mode(mode)
+    if m == TERNARY_B3:
+        return (26 * (K // GROUP) + 15) // 16 * 4  # 26 bytes per group, rows padded to 16 bytes
+    return K // (32 if m == BINARY else 16)
 
 
 def pack(codes, mode) -> np.ndarray:
-    """int8 codes [N,K] -> uint32 packed words [N, K/32] (binary) or [N, K/16]."""
+    """int8 codes [N,K] -> uint32 packed words [N, K/32] (binary), [N, K/16]
+    (INT2 ternary) or [N, 26*K/128 bytes rounded up to 16, as words] (base-3)."""
     c = _c(codes, np.int8)
     N, K = c.shape
     out = np.zeros((N, words_per_row(K, mode)), np.uint32)

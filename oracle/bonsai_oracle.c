@@ -30,6 +30,10 @@
  *
  * The bit layout of a packed word is this project's own format; the pages
  * only fix the number of bits per weight.  It is defined at oracle_pack.
+ * A third, denser ternary format (five trits per byte, 1.625 bits per
+ * weight; the pages' 1.71-bit figure is log2(3) + 16/128, and INT2 storage
+ * spends 2 bits) is this project's own too; it is defined at
+ * pack_b3_group.
  */
 #include <math.h>
 #include <pthread.h>
@@ -45,7 +49,9 @@
 
 #define MODE_BINARY 1
 #define MODE_TERNARY 2
+#define MODE_TERNARY_B3 3
 #define GROUP 128
+#define B3_GROUP_BYTES 26 /* ceil(128 / 5) */
 
 /* ---------------------------------------------------------------- FP16 -- */
 
@@ -103,20 +109,100 @@ void oracle_double_to_half_array(const double* x, int64_t n, uint16_t* out) {
 
 /* ------------------------------------------------------------- format -- */
 
-/* Weights per 32-bit word. */
+/* Weights per 32-bit word (binary and INT2 ternary). */
 static int per_word(int mode) { return mode == MODE_BINARY ? 32 : 16; }
 
 static int check_mode_shape(int64_t N, int64_t K, int mode) {
-  if (mode != MODE_BINARY && mode != MODE_TERNARY) return ORACLE_ERR_ARG;
+  if (mode != MODE_BINARY && mode != MODE_TERNARY && mode != MODE_TERNARY_B3) return ORACLE_ERR_ARG;
   if (N < 0 || K < 0) return ORACLE_ERR_SHAPE;
   if (K % GROUP != 0) return ORACLE_ERR_SHAPE;
   return ORACLE_OK;
 }
 
+/* Bytes of one packed row.  Base-3: 26 bytes per group of 128, the row
+ * padded with zero bytes to a multiple of 16. */
+static int64_t row_bytes(int64_t K, int mode) {
+  if (mode == MODE_TERNARY_B3) return (B3_GROUP_BYTES * (K / GROUP) + 15) / 16 * 16;
+  return K / per_word(mode) * 4;
+}
+
 /* Bytes of packed weights for an [N,K] matrix (scales not included). */
 int64_t oracle_packed_bytes(int64_t N, int64_t K, int mode) {
   if (check_mode_shape(N, K, mode) != ORACLE_OK) return -1;
-  return N * (K / per_word(mode)) * 4;
+  return N * row_bytes(K, mode);
+}
+
+/* Base-3 format.  A group of 128 ternary weights t[0..127] of one row
+ * becomes 26 bytes.  Byte j (0 <= j < 26) holds the five weights at
+ * positions j, j+26, j+52, j+78 and j+104 of the group as the base-3 number
+ *
+ *     byte[j] = sum_{i=0..4} q(26 i + j) * 3^(4-i),   q(k) = t[k] + 1,
+ *
+ * with q(k) = 0 for the two positions past the group (k = 128, 129, the
+ * last digit of bytes 24 and 25).  So the weight at position 26 i + j is the
+ * i-th base-3 digit of byte j, most significant first, minus one; bytes
+ * above 242 and non-zero padding digits are not codes.  Groups follow each
+ * other along K; a row's 26 * K/128 bytes are padded with zeros to a
+ * multiple of 16.  (Taking byte j's digits from positions 26 apart makes the
+ * same digit of bytes j and j+1 two neighbouring weights.) */
+static const int kPow3[5] = {81, 27, 9, 3, 1}; /* 3^(4-i) */
+
+static int pack_b3_group(const int8_t* t, uint8_t* out) {
+  for (int j = 0; j < B3_GROUP_BYTES; ++j) {
+    int value = 0;
+    for (int i = 0; i < 5; ++i) {
+      const int k = 26 * i + j;
+      int q = 0;
+      if (k < GROUP) {
+        if (t[k] < -1 || t[k] > 1) return ORACLE_ERR_BAD_CODE;
+        q = t[k] + 1;
+      }
+      value += q * kPow3[i];
+    }
+    out[j] = (uint8_t)value;
+  }
+  return ORACLE_OK;
+}
+
+static int unpack_b3_group(const uint8_t* in, int8_t* t) {
+  for (int j = 0; j < B3_GROUP_BYTES; ++j) {
+    int value = in[j];
+    if (value > 242) return ORACLE_ERR_BAD_CODE;
+    for (int i = 0; i < 5; ++i) {
+      const int q = (value / kPow3[i]) % 3;
+      const int k = 26 * i + j;
+      if (k < GROUP) t[k] = (int8_t)(q - 1);
+      else if (q != 0) return ORACLE_ERR_BAD_CODE;
+    }
+  }
+  return ORACLE_OK;
+}
+
+static int pack_b3(const int8_t* codes, int64_t N, int64_t K, uint8_t* packed) {
+  const int64_t rb = row_bytes(K, MODE_TERNARY_B3), groups = K / GROUP;
+  for (int64_t n = 0; n < N; ++n) {
+    uint8_t* row = packed + n * rb;
+    memset(row, 0, (size_t)rb);
+    for (int64_t g = 0; g < groups; ++g) {
+      int rc = pack_b3_group(codes + n * K + g * GROUP, row + g * B3_GROUP_BYTES);
+      if (rc != ORACLE_OK) return rc;
+    }
+  }
+  return ORACLE_OK;
+}
+
+static int unpack_b3(const uint8_t* packed, int64_t N, int64_t K, int8_t* codes) {
+  const int64_t rb = row_bytes(K, MODE_TERNARY_B3), groups = K / GROUP;
+  for (int64_t n = 0; n < N; ++n) {
+    const uint8_t* row = packed + n * rb;
+    for (int64_t g = 0; g < groups; ++g) {
+      int rc = unpack_b3_group(row + g * B3_GROUP_BYTES, codes + n * K + g * GROUP);
+      if (rc != ORACLE_OK) return rc;
+    }
+    for (int64_t b = groups * B3_GROUP_BYTES; b < rb; ++b)
+      if (row[b] != 0) return ORACLE_ERR_BAD_CODE; /* row padding */
+  }
+  return ORACLE_OK;
 }
 
 /* Bit position of weight i of a word.
@@ -139,6 +225,7 @@ static int ternary_low_bit(int i) { return 16 * (i & 1) + 14 - 2 * (i >> 1); }
 int oracle_pack(const int8_t* codes, int64_t N, int64_t K, int mode, uint32_t* packed) {
   int rc = check_mode_shape(N, K, mode);
   if (rc != ORACLE_OK) return rc;
+  if (mode == MODE_TERNARY_B3) return pack_b3(codes, N, K, (uint8_t*)packed);
   const int pw = per_word(mode);
   const int64_t words = K / pw;
   for (int64_t n = 0; n < N; ++n) {
@@ -167,6 +254,7 @@ int oracle_pack(const int8_t* codes, int64_t N, int64_t K, int mode, uint32_t* p
 int oracle_unpack(const uint32_t* packed, int64_t N, int64_t K, int mode, int8_t* codes) {
   int rc = check_mode_shape(N, K, mode);
   if (rc != ORACLE_OK) return rc;
+  if (mode == MODE_TERNARY_B3) return unpack_b3((const uint8_t*)packed, N, K, codes);
   const int pw = per_word(mode);
   const int64_t words = K / pw;
   for (int64_t n = 0; n < N; ++n) {
@@ -325,7 +413,7 @@ int oracle_gemm_entries(const uint16_t* A, const uint32_t* packed, const uint16_
                         double* absacc) {
   int rc = check_mode_shape(N, K, mode);
   if (rc != ORACLE_OK) return rc;
-  const int64_t words = K / per_word(mode);
+  const int64_t words = row_bytes(K, mode) / 4;
   int8_t* t = (int8_t*)malloc((size_t)(K > 0 ? K : 1));
   uint16_t* w16 = (uint16_t*)malloc((size_t)(K > 0 ? K : 1) * sizeof(uint16_t));
   if (!t || !w16) {

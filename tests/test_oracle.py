@@ -395,3 +395,87 @@ def test_stream_layer_lists():
     # 5 blocks x (4 image + 4 text linears) + 20 x 2 single-stream ones
     assert sum(1 for name, *_ in layers if ".img." in name) == 20
     assert sum(1 for name, *_ in layers if ".txt." in name) == 20
+
+
+# ------------------------------------------------ base-3 ternary format --
+# This project's denser format (five trits per byte; not on the pages, which
+# only state the 1.71-bit information figure and 2-bit INT2 storage): byte j
+# of a 128-weight group holds the weights at positions j, j+26, j+52, j+78,
+# j+104 as base-3 digits of t+1, most significant first; 26 bytes per group;
+# rows padded with zero bytes to a multiple of 16.
+
+def _b3_digits_lsb_first(b):
+    """Base-3 digits of b, least significant first, by repeated division."""
+    out = []
+    for _ in range(5):
+        b, r = divmod(b, 3)
+        out.append(r)
+    return out
+
+
+def test_b3_every_byte_value_at_every_position(oracle_mod):
+    """Exhaustive: each of the 243 byte values at each of the 26 byte
+    positions decodes to its base-3 digits at positions j + 26 i (digit i
+    counted from the most significant), zero bytes around it to t = -1."""
+    K = 128
+    for j in range(26):
+        rows = []
+        expected = []
+        for b in range(243):
+            d = _b3_digits_lsb_first(b)[::-1]  # most significant first
+            if j >= 24 and d[4] != 0:
+                continue  # the last digit of bytes 24, 25 is padding and must be zero
+            row = np.zeros(16 * 2, np.uint8)
+            row[j] = b
+            rows.append(row)
+            t = np.full(K, -1, np.int8)
+            for i in range(5):
+                if 26 * i + j < K:
+                    t[26 * i + j] = d[i] - 1
+            expected.append(t)
+        packed = np.stack(rows).view(np.uint32)
+        got = oracle_mod.unpack(packed, K, "ternary_b3")
+        assert np.array_equal(got, np.stack(expected)), j
+
+
+def test_b3_rejects_what_is_not_a_code(oracle_mod):
+    good = oracle_mod.pack(np.zeros((1, 128), np.int8), "ternary_b3")
+    for pos, value in [(3, 243), (0, 255), (24, 1), (25, 2), (26, 1), (31, 7)]:
+        bad = good.copy().view(np.uint8)
+        bad[0, pos] = value  # a byte above 242, a padding digit, row padding
+        with pytest.raises(oracle_mod.OracleError):
+            oracle_mod.unpack(bad.view(np.uint32), 128, "ternary_b3")
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.pack(np.full((1, 128), 2, np.int8), "ternary_b3")
+
+
+@pytest.mark.parametrize("K", [128, 256, 384, 1024, 3072])
+def test_b3_round_trip_and_size(oracle_mod, K):
+    rng = np.random.default_rng(K)
+    N = 7
+    codes = workloads.codes(rng, N, K, "ternary")
+    packed = oracle_mod.pack(codes, "ternary_b3")
+    assert np.array_equal(oracle_mod.unpack(packed, K, "ternary_b3"), codes)
+    row = -(-26 * (K // 128) // 16) * 16
+    assert oracle_mod.packed_bytes(N, K, "ternary_b3") == N * row == packed.nbytes
+    # 26 bytes per 128 weights: 1.625 bits, above log2(3) = 1.585 and below
+    # the 2 bits of INT2; with the FP16 scale per group 1.75 bits per weight.
+    assert 26 * 8 / 128 == 1.625
+    assert np.log2(3) < 1.625 < 2.0
+    assert (26 * 8 + 16) / 128 == 1.75
+
+
+def test_b3_weights_and_gemm_equal_int2_on_the_same_codes(oracle_mod):
+    """Same codes, two storage formats: the dequantised weights and the GEMM
+    (outputs, double sums, absolute sums) are identical."""
+    d = workloads.make(mode="ternary", M=9, N=33, K=640, seed=51)
+    p2 = oracle_mod.pack(d["codes"], "ternary")
+    p3 = oracle_mod.pack(d["codes"], "ternary_b3")
+    assert np.array_equal(oracle_mod.dequant(p2, d["scales"], 640, "ternary"),
+                          oracle_mod.dequant(p3, d["scales"], 640, "ternary_b3"))
+    o2, a2, s2 = oracle_mod.gemm(d["A"], p2, d["scales"], 640, "ternary")
+    o3, a3, s3 = oracle_mod.gemm(d["A"], p3, d["scales"], 640, "ternary_b3")
+    assert np.array_equal(o2, o3) and np.array_equal(a2, a3) and np.array_equal(s2, s3)
+    ms, ns = np.array([0, 8, 4]), np.array([32, 0, 17])
+    e3 = oracle_mod.gemm_entries(d["A"], p3, d["scales"], 640, "ternary_b3", ms, ns)
+    assert np.array_equal(e3[0], o2[ms, ns]) and np.array_equal(e3[1], a2[ms, ns])

@@ -23,6 +23,12 @@ MUTATIONS = {
                                   "static int binary_bit(int i) { return 16 * (1 - (i & 1)) + 15 - (i >> 1); }"),
     "scale row stride wrong": ("dequant_row(t + n * K, scales + n * (K / GROUP), K, w + n * K);",
                                "dequant_row(t + n * K, scales + n, K, w + n * K);"),
+    "base-3 digits read least significant first": ("const int q = (value / kPow3[i]) % 3;",
+                                                   "const int q = (value / kPow3[4 - i]) % 3;"),
+    "base-3 trit decoded with the wrong sign": ("if (k < GROUP) t[k] = (int8_t)(q - 1);",
+                                                "if (k < GROUP) t[k] = (int8_t)(1 - q);"),
+    "base-3 row pitch not padded": ("return (B3_GROUP_BYTES * (K / GROUP) + 15) / 16 * 16;",
+                                    "return B3_GROUP_BYTES * (K / GROUP);"),
 }
 
 
