@@ -136,15 +136,21 @@ int64_t oracle_packed_bytes(int64_t N, int64_t K, int mode) {
  * becomes 26 bytes.  Byte j (0 <= j < 26) holds the five weights at
  * positions j, j+26, j+52, j+78 and j+104 of the group as the base-3 number
  *
- *     byte[j] = sum_{i=0..4} q(26 i + j) * 3^(4-i),   q(k) = t[k] + 1,
+ *     v[j] = sum_{i=0..4} q(26 i + j) * 3^(4-i),   q(k) = t[k] + 1,
  *
  * with q(k) = 0 for the two positions past the group (k = 128, 129, the
- * last digit of bytes 24 and 25).  So the weight at position 26 i + j is the
- * i-th base-3 digit of byte j, most significant first, minus one; bytes
- * above 242 and non-zero padding digits are not codes.  Groups follow each
- * other along K; a row's 26 * K/128 bytes are padded with zeros to a
- * multiple of 16.  (Taking byte j's digits from positions 26 apart makes the
- * same digit of bytes j and j+1 two neighbouring weights.) */
+ * last digit of v[24] and v[25]), stored as the byte
+ *
+ *     byte[j] = ceil(256 * v[j] / 243),   so that   v[j] = floor(243 * byte[j] / 256).
+ *
+ * So the weight at position 26 i + j is the i-th base-3 digit of v[j], most
+ * significant first, minus one.  The 13 byte values that are no ceil(256 v /
+ * 243) and non-zero padding digits are not codes.  Groups follow each other
+ * along K; a row's 26 * K/128 bytes are padded with zeros to a multiple of
+ * 16.  (Storing 256 v / 243 rounded up makes the digits of a byte come out,
+ * most significant first, as the bits above 8 of repeated multiplications
+ * by 3; taking byte j's digits from positions 26 apart makes the same digit
+ * of bytes j and j+1 two neighbouring weights.) */
 static const int kPow3[5] = {81, 27, 9, 3, 1}; /* 3^(4-i) */
 
 static int pack_b3_group(const int8_t* t, uint8_t* out) {
@@ -159,15 +165,15 @@ static int pack_b3_group(const int8_t* t, uint8_t* out) {
       }
       value += q * kPow3[i];
     }
-    out[j] = (uint8_t)value;
+    out[j] = (uint8_t)((256 * value + 242) / 243); /* ceil(256 v / 243) */
   }
   return ORACLE_OK;
 }
 
 static int unpack_b3_group(const uint8_t* in, int8_t* t) {
   for (int j = 0; j < B3_GROUP_BYTES; ++j) {
-    int value = in[j];
-    if (value > 242) return ORACLE_ERR_BAD_CODE;
+    const int value = (243 * in[j]) / 256; /* floor(243 byte / 256) */
+    if ((256 * value + 242) / 243 != in[j]) return ORACLE_ERR_BAD_CODE;
     for (int i = 0; i < 5; ++i) {
       const int q = (value / kPow3[i]) % 3;
       const int k = 26 * i + j;

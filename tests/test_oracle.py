@@ -401,8 +401,14 @@ def test_stream_layer_lists():
 # This project's denser format (five trits per byte; not on the pages, which
 # only state the 1.71-bit information figure and 2-bit INT2 storage): byte j
 # of a 128-weight group holds the weights at positions j, j+26, j+52, j+78,
-# j+104 as base-3 digits of t+1, most significant first; 26 bytes per group;
-# rows padded with zero bytes to a multiple of 16.
+# j+104 as the base-3 digits of v = sum (t+1) 3^(4-i), most significant
+# first, stored as ceil(256 v / 243); 26 bytes per group; rows padded with
+# zero bytes to a multiple of 16.
+
+
+def _b3_byte(v):
+    """ceil(256 v / 243), exactly, in rational arithmetic."""
+    return math.ceil(Fraction(256 * v, 243))
 
 def _b3_digits_lsb_first(b):
     """Base-3 digits of b, least significant first, by repeated division."""
@@ -418,15 +424,17 @@ def test_b3_every_byte_value_at_every_position(oracle_mod):
     positions decodes to its base-3 digits at positions j + 26 i (digit i
     counted from the most significant), zero bytes around it to t = -1."""
     K = 128
+    zero = _b3_byte(0)
+    assert zero == 0  # all-zero padding bytes are valid (v = 0)
     for j in range(26):
         rows = []
         expected = []
-        for b in range(243):
-            d = _b3_digits_lsb_first(b)[::-1]  # most significant first
+        for v in range(243):
+            d = _b3_digits_lsb_first(v)[::-1]  # most significant first
             if j >= 24 and d[4] != 0:
                 continue  # the last digit of bytes 24, 25 is padding and must be zero
             row = np.zeros(16 * 2, np.uint8)
-            row[j] = b
+            row[j] = _b3_byte(v)
             rows.append(row)
             t = np.full(K, -1, np.int8)
             for i in range(5):
@@ -440,7 +448,12 @@ def test_b3_every_byte_value_at_every_position(oracle_mod):
 
 def test_b3_rejects_what_is_not_a_code(oracle_mod):
     good = oracle_mod.pack(np.zeros((1, 128), np.int8), "ternary_b3")
-    for pos, value in [(3, 243), (0, 255), (24, 1), (25, 2), (26, 1), (31, 7)]:
+    valid = {_b3_byte(v) for v in range(243)}
+    assert len(valid) == 243
+    not_codes = sorted(set(range(256)) - valid)
+    assert len(not_codes) == 13
+    cases = [(3, b) for b in not_codes] + [(24, _b3_byte(1)), (25, _b3_byte(2)), (26, 1), (31, 7)]
+    for pos, value in cases:
         bad = good.copy().view(np.uint8)
         bad[0, pos] = value  # a byte above 242, a padding digit, row padding
         with pytest.raises(oracle_mod.OracleError):

@@ -27,6 +27,8 @@ MUTATIONS = {
                                                    "const int q = (value / kPow3[4 - i]) % 3;"),
     "base-3 trit decoded with the wrong sign": ("if (k < GROUP) t[k] = (int8_t)(q - 1);",
                                                 "if (k < GROUP) t[k] = (int8_t)(1 - q);"),
+    "base-3 value stored rounded down": ("out[j] = (uint8_t)((256 * value + 242) / 243);",
+                                         "out[j] = (uint8_t)((256 * value) / 243);"),
     "base-3 row pitch not padded": ("return (B3_GROUP_BYTES * (K / GROUP) + 15) / 16 * 16;",
                                     "return B3_GROUP_BYTES * (K / GROUP);"),
 }
