@@ -136,13 +136,13 @@ def packed_bytes(N: int, K: int, mode) -> int:
 def words_per_row(K: int, mode) -> int:
     m = _mode(mode)
     if m == TERNARY_B3:
-        return (26 * (K // GROUP) + 15) // 16 * 4  # 26 bytes per group, rows padded to 16 bytes
+        return -(-(K // GROUP) // 4) * 28  # one 112-byte block (28 words) per 4 groups
     return K // (32 if m == BINARY else 16)
 
 
 def pack(codes, mode) -> np.ndarray:
     """int8 codes [N,K] -> uint32 packed words [N, K/32] (binary), [N, K/16]
-    (INT2 ternary) or [N, 26*K/128 bytes rounded up to 16, as words] (base-3)."""
+    (INT2 ternary) or [N, 28 * ceil(K/512)] (base-3: 112-byte blocks of 4 groups)."""
     c = _c(codes, np.int8)
     N, K = c.shape
     out = np.zeros((N, words_per_row(K, mode)), np.uint32)

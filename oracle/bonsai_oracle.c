@@ -30,10 +30,10 @@
  *
  * The bit layout of a packed word is this project's own format; the pages
  * only fix the number of bits per weight.  It is defined at oracle_pack.
- * A third, denser ternary format (five trits per byte, 1.625 bits per
- * weight; the pages' 1.71-bit figure is log2(3) + 16/128, and INT2 storage
- * spends 2 bits) is this project's own too; it is defined at
- * pack_b3_group.
+ * A third, denser ternary format (five trits per byte, 1.75 bits per weight
+ * with its alignment padding; the pages' 1.71-bit figure is log2(3) +
+ * 16/128, and INT2 storage spends 2 bits) is this project's own too; it is
+ * defined at pack_b3_group.
  */
 #include <math.h>
 #include <pthread.h>
@@ -51,7 +51,9 @@
 #define MODE_TERNARY 2
 #define MODE_TERNARY_B3 3
 #define GROUP 128
-#define B3_GROUP_BYTES 26 /* ceil(128 / 5) */
+#define B3_GROUP_BYTES 26  /* ceil(128 / 5) */
+#define B3_BLOCK_GROUPS 4  /* groups per 16-byte-aligned block */
+#define B3_BLOCK_BYTES 112 /* 4 x 26 data bytes + 8 zero bytes */
 
 /* ---------------------------------------------------------------- FP16 -- */
 
@@ -119,11 +121,16 @@ static int check_mode_shape(int64_t N, int64_t K, int mode) {
   return ORACLE_OK;
 }
 
-/* Bytes of one packed row.  Base-3: 26 bytes per group of 128, the row
- * padded with zero bytes to a multiple of 16. */
+/* Bytes of one packed row.  Base-3: one 112-byte block per 4 groups of 128
+ * (the last block of a row may hold fewer groups). */
 static int64_t row_bytes(int64_t K, int mode) {
-  if (mode == MODE_TERNARY_B3) return (B3_GROUP_BYTES * (K / GROUP) + 15) / 16 * 16;
+  if (mode == MODE_TERNARY_B3) return (K / GROUP + B3_BLOCK_GROUPS - 1) / B3_BLOCK_GROUPS * B3_BLOCK_BYTES;
   return K / per_word(mode) * 4;
+}
+
+/* Byte offset of group g within its row (base-3 format). */
+static int64_t b3_group_offset(int64_t g) {
+  return g / B3_BLOCK_GROUPS * B3_BLOCK_BYTES + g % B3_BLOCK_GROUPS * B3_GROUP_BYTES;
 }
 
 /* Bytes of packed weights for an [N,K] matrix (scales not included). */
@@ -146,8 +153,11 @@ int64_t oracle_packed_bytes(int64_t N, int64_t K, int mode) {
  * So the weight at position 26 i + j is the i-th base-3 digit of v[j], most
  * significant first, minus one.  The 13 byte values that are no ceil(256 v /
  * 243) and non-zero padding digits are not codes.  Groups follow each other
- * along K; a row's 26 * K/128 bytes are padded with zeros to a multiple of
- * 16.  (Storing 256 v / 243 rounded up makes the digits of a byte come out,
+ * along K in blocks of four: block b of a row is 112 bytes at offset 112 b,
+ * group 4b + r at byte 26 r of it; the block's last 8 bytes, and the group
+ * slots past the row's last group, are zero.  (The blocks keep every 4-group
+ * run on a 16-byte boundary, where a tensor-memory-access copy can start.
+ * Storing 256 v / 243 rounded up makes the digits of a byte come out,
  * most significant first, as the bits above 8 of repeated multiplications
  * by 3; taking byte j's digits from positions 26 apart makes the same digit
  * of bytes j and j+1 two neighbouring weights.) */
@@ -190,7 +200,7 @@ static int pack_b3(const int8_t* codes, int64_t N, int64_t K, uint8_t* packed) {
     uint8_t* row = packed + n * rb;
     memset(row, 0, (size_t)rb);
     for (int64_t g = 0; g < groups; ++g) {
-      int rc = pack_b3_group(codes + n * K + g * GROUP, row + g * B3_GROUP_BYTES);
+      int rc = pack_b3_group(codes + n * K + g * GROUP, row + b3_group_offset(g));
       if (rc != ORACLE_OK) return rc;
     }
   }
@@ -202,11 +212,15 @@ static int unpack_b3(const uint8_t* packed, int64_t N, int64_t K, int8_t* codes)
   for (int64_t n = 0; n < N; ++n) {
     const uint8_t* row = packed + n * rb;
     for (int64_t g = 0; g < groups; ++g) {
-      int rc = unpack_b3_group(row + g * B3_GROUP_BYTES, codes + n * K + g * GROUP);
+      int rc = unpack_b3_group(row + b3_group_offset(g), codes + n * K + g * GROUP);
       if (rc != ORACLE_OK) return rc;
     }
-    for (int64_t b = groups * B3_GROUP_BYTES; b < rb; ++b)
-      if (row[b] != 0) return ORACLE_ERR_BAD_CODE; /* row padding */
+    /* every byte outside the groups is padding and must be zero */
+    for (int64_t b = 0; b < rb; ++b) {
+      const int64_t r = b % B3_BLOCK_BYTES / B3_GROUP_BYTES, g = b / B3_BLOCK_BYTES * B3_BLOCK_GROUPS + r;
+      const int in_group = r < B3_BLOCK_GROUPS && g < groups;
+      if (!in_group && row[b] != 0) return ORACLE_ERR_BAD_CODE;
+    }
   }
   return ORACLE_OK;
 }

@@ -402,8 +402,8 @@ def test_stream_layer_lists():
 # only state the 1.71-bit information figure and 2-bit INT2 storage): byte j
 # of a 128-weight group holds the weights at positions j, j+26, j+52, j+78,
 # j+104 as the base-3 digits of v = sum (t+1) 3^(4-i), most significant
-# first, stored as ceil(256 v / 243); 26 bytes per group; rows padded with
-# zero bytes to a multiple of 16.
+# first, stored as ceil(256 v / 243); 26 bytes per group, four groups per
+# 112-byte block (8 zero bytes at its end), blocks along the row.
 
 
 def _b3_byte(v):
@@ -433,7 +433,7 @@ def test_b3_every_byte_value_at_every_position(oracle_mod):
             d = _b3_digits_lsb_first(v)[::-1]  # most significant first
             if j >= 24 and d[4] != 0:
                 continue  # the last digit of bytes 24, 25 is padding and must be zero
-            row = np.zeros(16 * 2, np.uint8)
+            row = np.zeros(112, np.uint8)
             row[j] = _b3_byte(v)
             rows.append(row)
             t = np.full(K, -1, np.int8)
@@ -452,7 +452,9 @@ def test_b3_rejects_what_is_not_a_code(oracle_mod):
     assert len(valid) == 243
     not_codes = sorted(set(range(256)) - valid)
     assert len(not_codes) == 13
-    cases = [(3, b) for b in not_codes] + [(24, _b3_byte(1)), (25, _b3_byte(2)), (26, 1), (31, 7)]
+    # bytes that are no code; a padding digit; an unused group slot; block padding
+    cases = [(3, b) for b in not_codes] + [(24, _b3_byte(1)), (25, _b3_byte(2)), (26, 1), (31, 7), (104, 1),
+                                            (111, 255)]
     for pos, value in cases:
         bad = good.copy().view(np.uint8)
         bad[0, pos] = value  # a byte above 242, a padding digit, row padding
@@ -469,13 +471,32 @@ def test_b3_round_trip_and_size(oracle_mod, K):
     codes = workloads.codes(rng, N, K, "ternary")
     packed = oracle_mod.pack(codes, "ternary_b3")
     assert np.array_equal(oracle_mod.unpack(packed, K, "ternary_b3"), codes)
-    row = -(-26 * (K // 128) // 16) * 16
+    row = 112 * -(-(K // 128) // 4)
     assert oracle_mod.packed_bytes(N, K, "ternary_b3") == N * row == packed.nbytes
-    # 26 bytes per 128 weights: 1.625 bits, above log2(3) = 1.585 and below
-    # the 2 bits of INT2; with the FP16 scale per group 1.75 bits per weight.
-    assert 26 * 8 / 128 == 1.625
-    assert np.log2(3) < 1.625 < 2.0
-    assert (26 * 8 + 16) / 128 == 1.75
+    # 112 bytes per 512 weights: 1.75 bits (1.625 of them trits), above
+    # log2(3) = 1.585 and below the 2 bits of INT2; with the FP16 scale per
+    # group 1.875 bits per weight against INT2's 2.125.
+    assert 112 * 8 / 512 == 1.75 and 26 * 8 / 128 == 1.625
+    assert np.log2(3) < 1.625 < 1.75 < 2.0
+    assert (112 * 8 + 4 * 16) / 512 == 1.875
+
+
+def test_b3_row_layout(oracle_mod):
+    """A row of 5 groups (two blocks) built by concatenation: per block the
+    26-byte groups in order, then zero bytes up to 112."""
+    rng = np.random.default_rng(5)
+    K = 640
+    codes = workloads.codes(rng, 3, K, "ternary")
+    for n in range(3):
+        groups = []
+        for g in range(K // 128):
+            t = codes[n, 128 * g:128 * (g + 1)].astype(int)
+            q = list(t + 1) + [0, 0]  # two padding positions, digit 0
+            groups.append(bytes(_b3_byte(sum(q[26 * i + j] * 3 ** (4 - i) for i in range(5))) for j in range(26)))
+        blocks = [b"".join(groups[b:b + 4]) for b in range(0, len(groups), 4)]
+        expected = b"".join(blk + bytes(112 - len(blk)) for blk in blocks)
+        got = oracle_mod.pack(codes, "ternary_b3")[n].tobytes()
+        assert got == expected, n
 
 
 def test_b3_weights_and_gemm_equal_int2_on_the_same_codes(oracle_mod):

@@ -29,8 +29,9 @@ MUTATIONS = {
                                                 "if (k < GROUP) t[k] = (int8_t)(1 - q);"),
     "base-3 value stored rounded down": ("out[j] = (uint8_t)((256 * value + 242) / 243);",
                                          "out[j] = (uint8_t)((256 * value) / 243);"),
-    "base-3 row pitch not padded": ("return (B3_GROUP_BYTES * (K / GROUP) + 15) / 16 * 16;",
-                                    "return B3_GROUP_BYTES * (K / GROUP);"),
+    "base-3 groups packed without blocks": (
+        "return g / B3_BLOCK_GROUPS * B3_BLOCK_BYTES + g % B3_BLOCK_GROUPS * B3_GROUP_BYTES;",
+        "return g * B3_GROUP_BYTES;"),
 }
 
 
