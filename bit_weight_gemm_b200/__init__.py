@@ -16,6 +16,7 @@ import torch
 
 BINARY = 1
 TERNARY = 2
+TERNARY_B3 = 3  # five trits per byte in 112-byte blocks of 4 groups (include/bonsai.h)
 GROUP = 128
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbonsai.so")
@@ -75,6 +76,8 @@ def _mode(mode) -> int:
         return BINARY
     if mode in (TERNARY, "ternary"):
         return TERNARY
+    if mode in (TERNARY_B3, "ternary_b3"):
+        return TERNARY_B3
     raise ValueError(f"unknown mode {mode!r}")
 
 
@@ -98,7 +101,10 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> ctypes.c_void_p:
 
 
 def words_per_row(K: int, mode) -> int:
-    return K // (32 if _mode(mode) == BINARY else 16)
+    m = _mode(mode)
+    if m == TERNARY_B3:
+        return -(-(K // GROUP) // 4) * 28
+    return K // (32 if m == BINARY else 16)
 
 
 def packed_bytes(N: int, K: int, mode) -> int:
@@ -110,7 +116,7 @@ def scale_bytes(N: int, K: int) -> int:
 
 
 def pack(codes: torch.Tensor, mode, out: torch.Tensor | None = None) -> torch.Tensor:
-    """int8 codes [N,K] on the device -> packed words (int32 view) [N, K/32] or [N, K/16]."""
+    """int8 codes [N,K] on the device -> packed words (int32 view) [N, words_per_row(K, mode)]."""
     N, K = codes.shape
     m = _mode(mode)
     if out is None:

@@ -20,7 +20,20 @@ constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s: far above any l
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool valid_mode(int mode) { return mode == BONSAI_BINARY || mode == BONSAI_TERNARY_INT2; }
+bool valid_mode(int mode) {
+  return mode == BONSAI_BINARY || mode == BONSAI_TERNARY_INT2 || mode == BONSAI_TERNARY_B3;
+}
+
+// Packed words of one row: K/32 (binary), K/16 (INT2), 28 per 4 groups (base-3).
+int64_t row_words(int64_t K, int mode) {
+  if (mode == BONSAI_TERNARY_B3) return (K / kGroup + kB3BlockGroups - 1) / kB3BlockGroups * (kB3BlockBytes / 4);
+  return K / (mode == BONSAI_BINARY ? 32 : 16);
+}
+
+// Tensor map of the packed weights: [N rows][row_words] uint32, copied in
+// boxes of one word stage (128 bytes of a row with 128-byte swizzling, or one
+// 112-byte base-3 block unswizzled) x 128 rows.
+bool make_weight_map(CUtensorMap* map, const void* packed, int N, int K, int mode);
 
 // K multiple of 128, sizes non-negative and small enough for 32-bit tile
 // coordinates and 64-bit byte counts.
@@ -157,6 +170,12 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void*
   return true;
 }
 
+bool make_weight_map(CUtensorMap* map, const void* packed, int N, int K, int mode) {
+  const bool b3 = mode == BONSAI_TERNARY_B3;
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, static_cast<uint64_t>(row_words(K, mode)), N,
+                  b3 ? kB3BlockBytes / 4 : 32, 128, b3 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // ------------------------------------------------------------------ GEMM --
 int sm_count() {
   static int count[64];
@@ -229,12 +248,9 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
   if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T, OCC>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
 
   CUtensorMap map_act, map_w, map_out;
-  const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
   if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, BLOCK_T, CU_TENSOR_MAP_SWIZZLE_128B))
     return BONSAI_ERR_CUDA;
-  if (!make_map(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, words_per_row, N, 32, T::kRows,
-                CU_TENSOR_MAP_SWIZZLE_128B))
-    return BONSAI_ERR_CUDA;
+  if (!make_weight_map(&map_w, packed, N, K, MODE)) return BONSAI_ERR_CUDA;
   const bool tma_store = (N % 8) == 0;
   if (tma_store) {
     if (!make_map(&map_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, out, N, M, T::kRows, BLOCK_T,
@@ -314,12 +330,9 @@ int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t
   auto kernel = lowbit_gemm_persistent_kernel<MODE>;
   if (smem_opt_in<lowbit_gemm_persistent_kernel<MODE>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
   CUtensorMap map_act, map_w;
-  const int words_per_row = K / (MODE == BONSAI_BINARY ? 32 : 16);
   if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, T::kBlockT, CU_TENSOR_MAP_SWIZZLE_128B))
     return BONSAI_ERR_CUDA;
-  if (!make_map(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, words_per_row, N, 32, T::kRows,
-                CU_TENSOR_MAP_SWIZZLE_128B))
-    return BONSAI_ERR_CUDA;
+  if (!make_weight_map(&map_w, packed, N, K, MODE)) return BONSAI_ERR_CUDA;
   PersistArgs args;
   args.scales = scales;
   args.out = out;
@@ -377,7 +390,9 @@ void consider(int M, int N, int K, Plan* best) {
   const int tiles = ((N + 127) / 128) * ((M + BLOCK_T - 1) / BLOCK_T);
   const TileCost c = tile_cost(BLOCK_T);
   const int sms = sm_count();
-  for (int ks = 1; ks <= 8 && ks <= groups; ++ks) {
+  // Base-3 ranges start on 4-group blocks: at most groups / 4 of them.
+  const int max_ks = MODE == BONSAI_TERNARY_B3 ? (groups / kB3BlockGroups > 1 ? groups / kB3BlockGroups : 1) : groups;
+  for (int ks = 1; ks <= 8 && ks <= max_ks; ++ks) {
     const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T, 1>(ks);
     if (per_wave <= 0) continue;
     const int waves = (tiles + per_wave - 1) / per_wave;
@@ -529,7 +544,7 @@ extern "C" {
 
 size_t bonsai_packed_bytes(int64_t N, int64_t K, int mode) {
   if (!valid_mode(mode) || check_shape(0, N, K) != BONSAI_OK) return 0;
-  return static_cast<size_t>(N) * static_cast<size_t>(K) / (mode == BONSAI_BINARY ? 8 : 4);
+  return static_cast<size_t>(N) * static_cast<size_t>(row_words(K, mode)) * 4;
 }
 
 size_t bonsai_scale_bytes(int64_t N, int64_t K) {
@@ -549,12 +564,17 @@ int bonsai_pack(const int8_t* codes, int64_t N, int64_t K, int mode, void* packe
   const unsigned zero = 0;
   if (cudaMemcpyToSymbolAsync(g_pack_bad_code, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return BONSAI_ERR_CUDA;
-  const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
-  const int grid = grid_for(words / 4, 256);
-  if (mode == BONSAI_BINARY)
-    pack_kernel<BONSAI_BINARY><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
-  else
-    pack_kernel<BONSAI_TERNARY_INT2><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
+  if (mode == BONSAI_TERNARY_B3) {
+    const int64_t blocks = N * (row_words(K, mode) / (kB3BlockBytes / 4));
+    pack_b3_kernel<<<grid_for(blocks, 256), 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), N, K);
+  } else {
+    const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
+    const int grid = grid_for(words / 4, 256);
+    if (mode == BONSAI_BINARY)
+      pack_kernel<BONSAI_BINARY><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
+    else
+      pack_kernel<BONSAI_TERNARY_INT2><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
+  }
   if ((rc = launch_status()) != BONSAI_OK) return rc;
   unsigned bad = 0;
   if (cudaMemcpyFromSymbolAsync(&bad, g_pack_bad_code, sizeof(bad), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
@@ -573,6 +593,11 @@ int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_
   if (!aligned16(packed) || !aligned16(scales) || !aligned16(w)) return BONSAI_ERR_ALIGN;
   if ((rc = check_device()) != BONSAI_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mode == BONSAI_TERNARY_B3) {
+    dequant_b3_kernel<<<grid_for(N * (K / kGroup), 256), 256, 0, st>>>(static_cast<const uint32_t*>(packed), scales, w,
+                                                                          N, K);
+    return launch_status();
+  }
   const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
   const int grid = grid_for(words, 256);
   if (mode == BONSAI_BINARY)
@@ -599,6 +624,7 @@ int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* sc
   if (!aligned16(A) || !aligned16(packed) || !aligned16(scales)) return BONSAI_ERR_ALIGN;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   if (mode == BONSAI_BINARY) return dispatch_gemm<BONSAI_BINARY>(A, packed, scales, m, n, k, out, st);
+  if (mode == BONSAI_TERNARY_B3) return dispatch_gemm<BONSAI_TERNARY_B3>(A, packed, scales, m, n, k, out, st);
   return dispatch_gemm<BONSAI_TERNARY_INT2>(A, packed, scales, m, n, k, out, st);
 }
 
@@ -621,6 +647,8 @@ int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const ui
   }
   if (mode == BONSAI_BINARY)
     return gemm_host_pipelined<BONSAI_BINARY>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
+  if (mode == BONSAI_TERNARY_B3)
+    return gemm_host_pipelined<BONSAI_TERNARY_B3>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
   return gemm_host_pipelined<BONSAI_TERNARY_INT2>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
 }
 
@@ -638,7 +666,9 @@ int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, in
   }
   if ((rc = check_device()) != BONSAI_OK) return rc;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-  const Plan p = mode == BONSAI_BINARY ? plan_gemm<BONSAI_BINARY>(m, n, k) : plan_gemm<BONSAI_TERNARY_INT2>(m, n, k);
+  const Plan p = mode == BONSAI_BINARY      ? plan_gemm<BONSAI_BINARY>(m, n, k)
+                 : mode == BONSAI_TERNARY_B3 ? plan_gemm<BONSAI_TERNARY_B3>(m, n, k)
+                                             : plan_gemm<BONSAI_TERNARY_INT2>(m, n, k);
   if (p.block_t == 0) return BONSAI_ERR_CUDA;
   *block_t = p.block_t;
   *ksplit = p.ksplit;

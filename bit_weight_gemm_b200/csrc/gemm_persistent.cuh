@@ -35,12 +35,14 @@ template <int MODE>
 struct PersistTile {
   static constexpr int kBlockT = 256;  // tokens per tile (MMA N)
   static constexpr int kRows = 128;    // weight rows per tile (MMA M)
-  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : 8;
-  static constexpr int kWGroups = 32 / kWordsPerGroup;  // groups per word stage
+  static constexpr bool kB3 = MODE == BONSAI_TERNARY_B3;
+  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : 8);  // held per group
+  static constexpr int kWGroups = kB3 ? kB3BlockGroups : 32 / kWordsPerGroup;    // groups per word stage
+  static constexpr int kWRowBytes = kB3 ? kB3BlockBytes : 128;                  // bytes of a row per stage
   static constexpr int kSliceBytes = kBlockT * 128;     // 256 rows x 64 FP16
   static constexpr int kActStageBytes = 2 * kSliceBytes;
   static constexpr int kActStages = 3;
-  static constexpr int kWStageBytes = kRows * 128;
+  static constexpr int kWStageBytes = kRows * kWRowBytes;
   static constexpr int kWStages = 2;
   static constexpr int kConvWarps = 16;  // four per TMEM lane quadrant
   static constexpr int kWarpsPerQuad = 4;
@@ -55,7 +57,7 @@ struct PersistTile {
   static constexpr int kNumBars = 2 * kActStages + 2 * kTStages + 2 * kWStages + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
-  static constexpr float kOutScale = MODE == BONSAI_BINARY ? 1.0f : 0.5f;
+  static constexpr float kOutScale = MODE == BONSAI_TERNARY_INT2 ? 0.5f : 1.0f;  // INT2 converts to 2ts
   // A converter warp takes the groups i = turn (mod 4) of every tile and
   // TMEM stage c % 4 of the running group count c: with four stages and
   // every tile's group count a multiple of four, warp `turn` always uses
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
         const uint32_t full = w_full0 + 8 * s;
         mbar_arrive_expect_tx_elected(full, T::kWStageBytes);
         tma_load_2d_elected(smem_addr(smem + T::kWOff + s * T::kWStageBytes), &tmap_w, full,
-                            j * T::kWGroups * T::kWordsPerGroup, n0);
+                            word_stage_x<MODE>(j * T::kWGroups), n0);
         last = wc;
       }
     }
@@ -254,10 +256,12 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
       if (!warp_wait(w_full0 + 8 * sw, (wc / WS) & 1, abort_flag, limit)) return false;
       if (!warp_wait(t_free0 + 8 * turn, ((c / TS) & 1) ^ 1, abort_flag, limit)) return false;
       tc_fence_after_sync();
-      const uint8_t* wrow = smem + T::kWOff + sw * T::kWStageBytes + row * 128;
+      const uint8_t* wrow = smem + T::kWOff + sw * T::kWStageBytes + row * T::kWRowBytes;
       const int pos = i % T::kWGroups;
       uint32_t words[T::kWordsPerGroup];
-      if (MODE == BONSAI_BINARY) {
+      if constexpr (T::kB3) {
+        b3_group_words(reinterpret_cast<const uint32_t*>(wrow), pos, words);
+      } else if (MODE == BONSAI_BINARY) {
         const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16 * (pos ^ (row & 7)));
         words[0] = q.x;
         words[1] = q.y;
@@ -278,7 +282,10 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
       __syncwarp();
       // Each warp reads kWGroups / 4 groups of a word stage; release after the last.
       if (lane == 0 && pos + T::kWarpsPerQuad >= T::kWGroups) mbar_arrive(w_empty0 + 8 * sw);
-      convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + turn * 64);
+      if constexpr (T::kB3)
+        convert_group_b3(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + turn * 64);
+      else
+        convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + turn * 64);
       tmem_store_wait();
       tc_fence_before_sync();
       __syncwarp();

@@ -67,7 +67,9 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
 template <int MODE, int BLOCK_T, int OCC = 1>
 struct GemmTile {
   static constexpr int kRows = 128;  // weight rows per tile (MMA M)
-  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : 8;
+  static constexpr bool kB3 = MODE == BONSAI_TERNARY_B3;
+  // Words a converter holds per group: 4 binary, 8 INT2, 7 base-3 (26 bytes).
+  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : 8);
   static constexpr int kSliceBytes = BLOCK_T * 128;       // BLOCK_T rows x 64 FP16
   static constexpr int kActStageBytes = 2 * kSliceBytes;  // 128 K per stage
   // Activation stages: as many as fit next to the word ring and the scales,
@@ -77,8 +79,14 @@ struct GemmTile {
                : (BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : (96 * 1024) / kActStageBytes));
   // A word stage is 128 bytes of every row: 4 ternary or 8 binary groups,
   // one TMA box with 128-byte swizzling.
-  static constexpr int kWGroups = 32 / kWordsPerGroup;
-  static constexpr int kWStageBytes = kRows * 128;
+  // Base-3: one 112-byte block (4 groups) of every row per stage, without
+  // swizzling (a 112-byte box is not a 128-byte swizzle span).
+  static constexpr int kWGroups = kB3 ? kB3BlockGroups : 32 / kWordsPerGroup;
+  static constexpr int kWRowBytes = kB3 ? kB3BlockBytes : 128;
+  static constexpr int kWStageBytes = kRows * kWRowBytes;
+  // Split-K ranges of base-3 weights start on block boundaries (TMA copies
+  // start on 16-byte boundaries).
+  static constexpr int kGroupAlign = kB3 ? kB3BlockGroups : 1;
   // Small token tiles are bandwidth-bound: enough word stages to keep every
   // load of a split-K CTA in flight at once.
   static constexpr int kWStages = (OCC == 2 || BLOCK_T >= 256) ? 2 : 4;
@@ -126,7 +134,7 @@ struct GemmTile {
   // keeps it off the SM.
   static constexpr int kSmemBytes = (OCC == 1 && kSmemNeeded < 116 * 1024) ? 116 * 1024 : kSmemNeeded;
 
-  static constexpr float kOutScale = MODE == BONSAI_BINARY ? 1.0f : 0.5f;
+  static constexpr float kOutScale = MODE == BONSAI_TERNARY_INT2 ? 0.5f : 1.0f;  // INT2 converts to 2ts
   static_assert(BLOCK_T % 16 == 0 && BLOCK_T >= 16 && BLOCK_T <= 256, "MMA N for M=128");
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(OCC == 1 || OCC == 2, "one or two CTAs per SM");
@@ -169,6 +177,44 @@ __device__ __forceinline__ void convert_group(const uint32_t* words, uint32_t s2
       tmem_store_8(taddr + j * 8, v);
     }
   }
+}
+
+// Base-3: the group's 26 bytes (7 words from b3_group_words) -> 64 TMEM
+// columns of FP16 pairs t*s; column 13 i + p holds digit i of byte pair p,
+// i.e. the weights 26 i + 2p and 26 i + 2p + 1.
+__device__ __forceinline__ void convert_group_b3(const uint32_t* words, uint32_t s2, uint32_t taddr) {
+  uint32_t y[13];
+#pragma unroll
+  for (int p = 0; p < 13; ++p) y[p] = b3_byte_pair(words, p);
+  uint32_t v[8];
+#pragma unroll
+  for (int i = 0; i < 5; ++i)
+#pragma unroll
+    for (int p = 0; p < 13; ++p) {
+      const int c = 13 * i + p;
+      if (c < 64) {
+        v[c & 7] = hmul2_bits(b3_next_t_pair(y[p]), s2);
+        if ((c & 7) == 7) tmem_store_8(taddr + (c - 7), v);
+      }
+    }
+}
+
+// First word (uint32 x coordinate of the packed-weight tensor map) of the
+// word stage that starts at group g0.
+template <int MODE>
+__device__ __forceinline__ int word_stage_x(int g0) {
+  if (MODE == BONSAI_TERNARY_B3) return g0 / kB3BlockGroups * (kB3BlockBytes / 4);
+  return g0 * (MODE == BONSAI_BINARY ? 4 : 8);
+}
+
+// Boundary z of a split of `groups` into `ks` ranges, on multiples of ALIGN
+// (nearest); the caller keeps ks <= groups / ALIGN so that no range is empty.
+template <int ALIGN>
+__device__ __forceinline__ int split_bound(int z, int groups, int ks) {
+  if (z >= ks) return groups;
+  const int x = static_cast<int>(static_cast<int64_t>(z) * groups / ks);
+  const int r = (x + ALIGN / 2) / ALIGN * ALIGN;
+  return r < groups ? r : groups;
 }
 
 // A wait the whole warp agrees on: every lane waits, and the warp goes on
@@ -237,8 +283,8 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
   const int n0 = blockIdx.x * T::kRows;
   const int m0 = blockIdx.y * BLOCK_T;
   const int groups = args.K / kGroup;
-  const int g_begin = static_cast<int>(static_cast<int64_t>(blockIdx.z) * groups / args.ksplit);
-  const int g_end = static_cast<int>(static_cast<int64_t>(blockIdx.z + 1) * groups / args.ksplit);
+  const int g_begin = split_bound<T::kGroupAlign>(static_cast<int>(blockIdx.z), groups, args.ksplit);
+  const int g_end = split_bound<T::kGroupAlign>(static_cast<int>(blockIdx.z) + 1, groups, args.ksplit);
   const int ng = g_end - g_begin;
   const uint64_t limit = args.wait_limit_ns;
 
@@ -274,7 +320,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
     // still run (they are read-only here; the copies into shared memory
     // follow griddep_wait).
     const int nw = (ng + T::kWGroups - 1) / T::kWGroups;
-    for (int i = 0; i < nw; ++i) tma_prefetch_l2_2d(&tmap_w, (g_begin + i * T::kWGroups) * T::kWordsPerGroup, n0);
+    for (int i = 0; i < nw; ++i) tma_prefetch_l2_2d(&tmap_w, word_stage_x<MODE>(g_begin + i * T::kWGroups), n0);
     if (args.scale_box > 0) tma_prefetch_l2_2d(&tmap_s, g_begin & ~7, n0);
   }
   if (warp == 1) {
@@ -331,7 +377,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
       const uint32_t full = w_full0 + 8 * s;
       mbar_arrive_expect_tx_elected(full, T::kWStageBytes);
       tma_load_2d_elected(smem_addr(smem + T::kWOff + s * T::kWStageBytes), &tmap_w, full,
-                          (g_begin + i * T::kWGroups) * T::kWordsPerGroup, n0);
+                          word_stage_x<MODE>(g_begin + i * T::kWGroups), n0);
       issued = i + 1;
     }
     if (*abort_flag) {
@@ -439,9 +485,11 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
       const uint8_t* wstage = smem + T::kWOff + sw * T::kWStageBytes;
       // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
       const int pos = i % T::kWGroups;
-      const uint8_t* wrow = wstage + row * 128;
+      const uint8_t* wrow = wstage + row * T::kWRowBytes;
       uint32_t words[T::kWordsPerGroup];
-      if (MODE == BONSAI_BINARY) {
+      if constexpr (T::kB3) {
+        b3_group_words(reinterpret_cast<const uint32_t*>(wrow), pos, words);
+      } else if (MODE == BONSAI_BINARY) {
         const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16 * (pos ^ (row & 7)));
         words[0] = q.x;
         words[1] = q.y;
@@ -466,7 +514,10 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
       // may lack some warps' arrivals.
       const int stage_end = (wj + 1) * T::kWGroups < ng ? (wj + 1) * T::kWGroups : ng;
       if (lane == 0 && i + kStep >= stage_end) mbar_arrive(w_empty0 + 8 * sw);
-      convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
+      if constexpr (T::kB3)
+        convert_group_b3(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
+      else
+        convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
       tmem_store_wait();
       tc_fence_before_sync();
       __syncwarp();

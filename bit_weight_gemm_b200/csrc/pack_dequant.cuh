@@ -122,4 +122,129 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
   }
 }
 
+// ------------------------------------------------- base-3 ternary format --
+// (bonsai.h.)  A group's byte j holds the trits at group positions j, j+26,
+// j+52, j+78, j+104 as y = ceil(256 v / 243), v their base-3 number
+// (digits t+1, most significant first).  y / 256 is v / 243 plus less than
+// 1/243, so multiplying y by 3 puts the next digit in bits 8-9 and leaves
+// the rest of the fraction in the low byte, exactly, five times.  Two bytes
+// j and j+1 side by side as 16-bit lanes step together; their same digit is
+// the pair of neighbouring weights (26 i + j, 26 i + j + 1).
+constexpr int kB3GroupBytes = 26;
+constexpr int kB3BlockGroups = 4;
+constexpr int kB3BlockBytes = 112;  // 4 x 26 bytes + 8 zero bytes
+constexpr uint32_t kB3Minus1025 = 0xE401E401u;  // FP16 -1025 in both halves
+
+// Bytes 2p and 2p+1 of the group's (aligned) words as the 16-bit lanes of one
+// register.
+__device__ __forceinline__ uint32_t b3_byte_pair(const uint32_t* w, int p) {
+  return __byte_perm(w[p >> 1], 0u, (p & 1) ? 0x4342u : 0x4140u);
+}
+
+// Steps a byte pair to its next digit pair and returns (t0, t1) as FP16:
+// the digits d land under FP16's exponent of 1024 (byte 0x64 above them)
+// and 1024 + d - 1025 = t exactly.
+__device__ __forceinline__ uint32_t b3_next_t_pair(uint32_t& y) {
+  const uint32_t t3 = y * 3u;
+  y = t3 & 0x00FF00FFu;
+  const uint32_t magic = __byte_perm(t3, 0x64646464u, 0x4341u);  // (1024 + d0, 1024 + d1)
+  uint32_t t;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(t) : "r"(magic), "r"(kB3Minus1025));
+  return t;
+}
+
+// Loads the 26 bytes of group slot r (0..3) of a row's block as 7 words
+// aligned to the group's first byte (slots 1 and 3 start 2 bytes into a word).
+__device__ __forceinline__ void b3_group_words(const uint32_t* block, int r, uint32_t* w) {
+  const int w0 = (kB3GroupBytes * r) >> 2;
+  uint32_t raw[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) raw[k] = block[w0 + k];
+  const bool odd = (r & 1) != 0;
+#pragma unroll
+  for (int k = 0; k < 7; ++k) w[k] = odd ? __funnelshift_r(raw[k], raw[k + 1], 16) : raw[k];
+}
+
+// Packs the codes of one row's block b (groups 4b .. 4b+3 that exist) into
+// 112 bytes.  One thread per block; codes are read as 16-byte loads.
+__global__ void __launch_bounds__(256) pack_b3_kernel(const int8_t* __restrict__ codes, uint32_t* __restrict__ packed,
+                                                      int64_t N, int64_t K) {
+  const int64_t groups = K / kGroup;
+  const int64_t blocks_per_row = (groups + kB3BlockGroups - 1) / kB3BlockGroups;
+  const int64_t total = N * blocks_per_row;
+  bool ok = true;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = idx / blocks_per_row, b = idx - n * blocks_per_row;
+    uint32_t out[kB3BlockBytes / 4] = {};
+#pragma unroll
+    for (int r = 0; r < kB3BlockGroups; ++r) {
+      const int64_t g = b * kB3BlockGroups + r;
+      if (g >= groups) break;
+      const uint4* src = reinterpret_cast<const uint4*>(codes + n * K + g * kGroup);
+      uint32_t c[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = __ldg(src + i);
+        c[4 * i] = v.x;
+        c[4 * i + 1] = v.y;
+        c[4 * i + 2] = v.z;
+        c[4 * i + 3] = v.w;
+      }
+#pragma unroll
+      for (int j = 0; j < kB3GroupBytes; ++j) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+          const int k = 26 * i + j;
+          uint32_t q = 0;  // positions past the group: digit 0
+          if (k < kGroup) {
+            q = ((c[k >> 2] >> (8 * (k & 3))) + 1u) & 0xFFu;  // t + 1 for t in {-1, 0, +1}
+            ok &= q <= 2u;
+          }
+          v = 3u * v + q;
+        }
+        const uint32_t y = (256u * v + 242u) / 243u;  // ceil(256 v / 243)
+        const int byte = kB3GroupBytes * r + j;
+        out[byte >> 2] |= (y & 0xFFu) << (8 * (byte & 3));
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(packed) + idx * (kB3BlockBytes / 16);
+#pragma unroll
+    for (int i = 0; i < kB3BlockBytes / 16; ++i) dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+  }
+  if (!__all_sync(0xffffffffu, ok) && lane_id() == 0) atomicOr(&g_pack_bad_code, 1u);
+}
+
+// Exact dequantisation of the base-3 format: one thread per (row, group);
+// t comes out of the digit step as an exact FP16 -1, +0 or +1 and one IEEE
+// FP16 multiply by the scale gives t * s.
+__global__ void __launch_bounds__(256) dequant_b3_kernel(const uint32_t* __restrict__ packed,
+                                                         const uint16_t* __restrict__ scales,
+                                                         uint16_t* __restrict__ w, int64_t N, int64_t K) {
+  const int64_t groups = K / kGroup;
+  const int64_t row_words = (groups + kB3BlockGroups - 1) / kB3BlockGroups * (kB3BlockBytes / 4);
+  const int64_t total = N * groups;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = idx / groups, g = idx - n * groups;
+    const uint32_t* block = packed + n * row_words + g / kB3BlockGroups * (kB3BlockBytes / 4);
+    uint32_t words[7];
+    b3_group_words(block, static_cast<int>(g % kB3BlockGroups), words);
+    const uint32_t s = __ldg(scales + n * groups + g);
+    const uint32_t s2 = s | (s << 16);
+    uint32_t y[13];
+#pragma unroll
+    for (int p = 0; p < 13; ++p) y[p] = b3_byte_pair(words, p);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(w + n * K + g * kGroup);  // FP16 pairs: weights 2c, 2c+1
+#pragma unroll
+    for (int i = 0; i < 5; ++i)
+#pragma unroll
+      for (int p = 0; p < 13; ++p) {
+        const int c = 13 * i + p;
+        if (c < kGroup / 2) dst[c] = hmul2_bits(b3_next_t_pair(y[p]), s2);
+      }
+  }
+}
+
 }  // namespace bonsai

@@ -21,6 +21,14 @@
  *   binary : bit 16h + 15 - p; 1 means t = -1, 0 means t = +1;
  *   ternary: bits 16h + 14 - 2p (magnitude) and 16h + 15 - 2p (sign);
  *            t = 0 -> 00, t = +1 -> 01, t = -1 -> 11; 10 is not a code.
+ * Base-3 ternary (BONSAI_TERNARY_B3, denser: 1.75 bits per weight against
+ * INT2's 2): a row is a run of 112-byte blocks, one per 4 groups of 128
+ * weights along K (28 * ceil(K/512) words); group 4b + r sits at byte
+ * 112 b + 26 r; the block's last 8 bytes and group slots past the row's last
+ * group are zero.  Byte j of a group holds the weights at group positions
+ * j, j+26, j+52, j+78, j+104 as v = sum_i (t+1) 3^(4-i) (positions past 127
+ * count as t+1 = 0), stored as the byte ceil(256 v / 243); the 13 other byte
+ * values are not codes.
  * Scales: FP16 [N, K/128], row-major.  Activations: FP16 [M, K], row-major.
  * Output: FP16 [M, N], row-major.  FP16 values travel as uint16_t bits.
  *
@@ -47,7 +55,8 @@ extern "C" {
 
 typedef enum {
   BONSAI_BINARY = 1,       /* t in {-1,+1}, 1 bit per weight */
-  BONSAI_TERNARY_INT2 = 2  /* t in {-1,0,+1}, 2 bits per weight */
+  BONSAI_TERNARY_INT2 = 2, /* t in {-1,0,+1}, 2 bits per weight */
+  BONSAI_TERNARY_B3 = 3    /* t in {-1,0,+1}, five per byte: 1.75 bits per weight */
 } bonsai_mode;
 
 typedef enum {
@@ -61,8 +70,9 @@ typedef enum {
   BONSAI_ERR_TIMEOUT = 7      /* a kernel gave up a bounded wait (see bonsai_get_device_error) */
 } bonsai_status;
 
-/* Bytes of packed weights for an [N,K] weight: N*K/8 (binary) or N*K/4
- * (ternary).  Returns 0 for an invalid mode or shape. */
+/* Bytes of packed weights for an [N,K] weight: N*K/8 (binary), N*K/4
+ * (INT2 ternary) or N*112*ceil(K/512) (base-3 ternary).  Returns 0 for an
+ * invalid mode or shape. */
 size_t bonsai_packed_bytes(int64_t N, int64_t K, int mode);
 
 /* Bytes of the FP16 scales for an [N,K] weight: 2*N*K/128. */
@@ -87,10 +97,11 @@ int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_
  * A: FP16 [M,K]; packed/scales: as above for an [N,K] weight; out: FP16
  * [M,N].  Products are formed exactly and summed in FP32 on the tensor
  * cores, then rounded once to FP16 (nearest even).  Scales must be finite
- * with |s| < 32768 for ternary weights (the kernel forms 2*s*t in FP16);
- * outside that range the result is unspecified.  out must not overlap A,
- * packed or scales.  A packed field with the pattern 10 (not a ternary
- * code) contributes zero. */
+ * with |s| < 32768 for INT2 ternary weights (the kernel forms 2*s*t in
+ * FP16); outside that range the result is unspecified.  out must not
+ * overlap A, packed or scales.  An INT2 field with the pattern 10 (not a
+ * ternary code) contributes zero; a base-3 byte that is not a code gives
+ * unspecified values for its five weights. */
 int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int64_t M,
                        int64_t N, int64_t K, int mode, uint16_t* out, void* stream);
 

@@ -62,13 +62,15 @@ def test_sizes(lib):
     assert bw.packed_bytes(3072, 9216, "binary") == 3072 * 9216 // 8
     assert bw.scale_bytes(3072, 9216) == 3072 * 72 * 2
     assert bw.packed_bytes(8, 100, "ternary") == 0  # partial group
-    assert lib.bonsai_packed_bytes(8, 128, 3) == 0  # unknown mode
+    assert bw.packed_bytes(3072, 9216, "ternary_b3") == 3072 * 112 * (9216 // 512)  # 112-byte blocks of 4 groups
+    assert bw.packed_bytes(8, 640, "ternary_b3") == 8 * 112 * 2  # a partial last block still takes 112 bytes
+    assert lib.bonsai_packed_bytes(8, 128, 4) == 0  # unknown mode
     assert lib.bonsai_packed_bytes(-1, 128, 2) == 0
 
 
 def test_argument_errors_before_any_device_work(lib):
     P = None
-    assert lib.bonsai_pack(P, 4, 128, 3, P, P) == 1  # mode
+    assert lib.bonsai_pack(P, 4, 128, 4, P, P) == 1  # mode
     assert lib.bonsai_pack(P, 4, 100, 2, P, P) == 2  # K % 128
     assert lib.bonsai_pack(P, -4, 128, 2, P, P) == 2
     assert lib.bonsai_pack(P, 0, 128, 2, P, P) == 0  # empty: no-op

@@ -17,6 +17,7 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 RTOL = 1e-3
+MODES = ["binary", "ternary", "ternary_b3"]  # ternary_b3: the same codes in the base-3 storage format
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -74,7 +75,7 @@ def assert_gemm_close(oracle_mod, got_bits, ref_bits, absacc, label):
 PACK_SHAPES = [(1, 128), (37, 384), (256, 256), (129, 1152), (1000, 3072)]
 
 
-@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("N,K", PACK_SHAPES)
 def test_pack_bit_exact(oracle_mod, mode, N, K):
     d = workloads.make(mode=mode, M=1, N=N, K=K, seed=N * 7 + K)
@@ -83,7 +84,8 @@ def test_pack_bit_exact(oracle_mod, mode, N, K):
     assert np.array_equal(to_u32(got), ref)
 
 
-@pytest.mark.parametrize("mode,bad", [("ternary", 2), ("ternary", -2), ("binary", 0), ("binary", 3)])
+@pytest.mark.parametrize("mode,bad", [("ternary", 2), ("ternary", -2), ("binary", 0), ("binary", 3),
+                                      ("ternary_b3", 2), ("ternary_b3", -128)])
 def test_pack_reports_bad_codes(mode, bad):
     c = np.ones((64, 256), np.int8)
     c[63, 255] = bad
@@ -95,7 +97,7 @@ def test_pack_reports_bad_codes(mode, bad):
 
 
 # --------------------------------------------------------------- dequant
-@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("N,K", PACK_SHAPES)
 def test_dequant_bit_exact(oracle_mod, mode, N, K):
     d = workloads.make(mode=mode, M=1, N=N, K=K, seed=N * 3 + K)
@@ -105,7 +107,7 @@ def test_dequant_bit_exact(oracle_mod, mode, N, K):
     assert np.all(nan_aware_equal(to_u16(got), ref))
 
 
-@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("mode", MODES)
 def test_dequant_every_scale_pattern(oracle_mod, mode):
     N, K = 65536, 128
     rng = np.random.default_rng(12)
@@ -142,7 +144,7 @@ def test_gemm_ternary_tiny_config(oracle_mod):
     assert_gemm_close(oracle_mod, got, ref, absacc, p.name)
 
 
-@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("M,N,K", SMALL_SHAPES)
 def test_gemm_ragged_shapes(oracle_mod, mode, M, N, K):
     got, ref, absacc = _gemm_case(oracle_mod, mode, M, N, K, seed=M * 31 + N * 7 + K)
@@ -171,7 +173,9 @@ def _sample_positions(M, N, block_t, count, seed):
 
 
 FULL = [workloads.TERNARY_MLP_UP_4608, workloads.TERNARY_MLP_DOWN_4608, workloads.TERNARY_QKV_4608,
-        workloads.TERNARY_MLP_DOWN_16, workloads.TERNARY_QKV_16]
+        workloads.TERNARY_MLP_DOWN_16, workloads.TERNARY_QKV_16,
+        workloads.Problem("base-3 ternary MLP-up M=4608", "ternary_b3", 4608, 9216, 3072, 1003),
+        workloads.Problem("base-3 ternary MLP-down M=16", "ternary_b3", 16, 3072, 9216, 1014)]
 
 
 @pytest.mark.parametrize("problem", FULL, ids=[p.name for p in FULL])
@@ -227,6 +231,8 @@ def test_plan_in_a_fresh_process_matches_launch():
 # N odd in the third case.
 LARGE_M_SHAPES = [
     ("ternary", 1357, 3880, 512, True),
+    ("ternary_b3", 1357, 3880, 512, True),
+    ("ternary_b3", 700, 6376, 1152, False),
     ("binary", 700, 6376, 1024, True),
     ("ternary", 513, 9999, 1024, True),
     ("ternary", 1357, 3880, 640, False),
@@ -244,7 +250,7 @@ def test_gemm_large_m_full(oracle_mod, mode, M, N, K, persistent):
 
 
 # ------------------------------------------------------------ invariants
-@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("M", [16, 200])
 def test_gemm_sign_symmetry_bitwise(mode, M):
     d = workloads.make(mode=mode, M=M, N=256, K=512, seed=M + 5)
@@ -255,7 +261,7 @@ def test_gemm_sign_symmetry_bitwise(mode, M):
     assert torch.equal(neg, -pos)
 
 
-@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("mode", MODES)
 def test_gemm_power_of_two_scaling_bitwise(mode):
     d = workloads.make(mode=mode, M=100, N=384, K=384, seed=77)
     A = dev(d["A"].view(np.int16), torch.float16)
@@ -270,7 +276,7 @@ def test_gemm_power_of_two_scaling_bitwise(mode):
     assert torch.equal(two[normal], one[normal] * 2)
 
 
-@pytest.mark.parametrize("mode", ["binary", "ternary"])
+@pytest.mark.parametrize("mode", MODES)
 def test_gemm_all_ones_closed_form(oracle_mod, mode):
     N, K = 256, 1024
     rng = np.random.default_rng(99)
@@ -317,7 +323,8 @@ def test_gemm_matches_dequant_then_torch_matmul():
 # back-to-back launches give the race its chances.
 @pytest.mark.parametrize("mode,M,N,K", [("ternary", 16, 3072, 12288), ("ternary", 32, 3072, 12288),
                                         ("ternary", 64, 3072, 12288), ("ternary", 64, 9216, 3072),
-                                        ("binary", 64, 3072, 12288), ("ternary", 128, 3072, 12288)])
+                                        ("binary", 64, 3072, 12288), ("ternary", 128, 3072, 12288),
+                                        ("ternary_b3", 16, 3072, 12288), ("ternary_b3", 64, 9216, 3072)])
 def test_narrow_tiles_repeated_launches(oracle_mod, mode, M, N, K):
     d = workloads.make(mode=mode, M=M, N=N, K=K, seed=M + N + K)
     ref_packed, packed, A, scales = gpu_inputs(d, oracle_mod)

@@ -27,7 +27,7 @@ GROUP = 128
 @dataclass(frozen=True)
 class Problem:
     name: str
-    mode: str  # "binary" | "ternary"
+    mode: str  # "binary" | "ternary" (INT2) | "ternary_b3" (base-3 storage of the same codes)
     M: int
     N: int
     K: int
@@ -108,7 +108,7 @@ def codes(rng: np.random.Generator, N: int, K: int, mode: str) -> np.ndarray:
     u = rng.random((N, K), dtype=np.float64)
     if mode == "binary":
         return np.where(u < 0.5, 1, -1).astype(np.int8)
-    if mode == "ternary":
+    if mode in ("ternary", "ternary_b3"):  # one code alphabet, two storage formats
         return np.where(u < 0.3, -1, np.where(u < 0.7, 0, 1)).astype(np.int8)
     raise ValueError(mode)
 
