@@ -62,10 +62,17 @@ def flops(p) -> int:
     return 2 * p.M * p.N * p.K
 
 
+def packed_weight_bytes(mode, N, K) -> int:
+    """Packed weight bytes: K/8 (binary), K/4 (INT2) or 112 per 512 weights
+    (base-3 blocks) per row."""
+    if mode == "ternary_b3":
+        return N * 112 * -(-(K // 128) // 4)
+    return N * K // (8 if mode == "binary" else 4)
+
+
 def algorithmic_bytes(p) -> int:
     """Packed weights + FP16 scales + FP16 activations in + FP16 output."""
-    wbytes = p.N * p.K // (8 if p.mode == "binary" else 4)
-    return wbytes + 2 * p.N * (p.K // 128) + 2 * p.M * p.K + 2 * p.M * p.N
+    return packed_weight_bytes(p.mode, p.N, p.K) + 2 * p.N * (p.K // 128) + 2 * p.M * p.K + 2 * p.M * p.N
 
 
 def load_peaks():
@@ -366,8 +373,10 @@ def run_bonsai(args):
         stack += [time_stack(torch, bw, None, "ternary", 20, 3, streams=st) for st in ((4096, 512), (1024, 512))]
         stack += [time_stack(torch, bw, m, "binary", 20, 3) for m in (4608, 1024)]
     cublas = None
+    formats = None
     if not args.no_extras and not args.small_only:
         cublas = cublas_fp16_same_run(torch)
+        formats = time_formats(torch, bw, args, dist, peaks, peaks_kind)
 
     if dist is not None:
         dist.barrier()
@@ -395,6 +404,7 @@ def run_bonsai(args):
                 "cpu_baseline": cpu,
                 "small_m": small,
                 "stack": stack,
+                "formats": formats,
             }
             print(json.dumps(line), flush=True)
     if dist is not None:
@@ -457,6 +467,26 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
                          "frac": achieved / peak, "traffic": ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}"),
                          "algorithmic_bytes_per_launch": nbytes, "peak_source": f"{peaks_kind} hbm copy"},
             "gpu_launches": steps}
+
+
+def time_formats(torch, bw, args, dist, peaks, peaks_kind):
+    """The headline and the M=16 workloads with the same ternary codes stored
+    in the base-3 format (1.75 bits per weight against INT2's 2): TFLOP/s at
+    M=4608 and GB/s of algorithmic bytes (fewer packed bytes) at M=16."""
+    out = []
+    for base, sets_n, unit in ((WORKLOAD, args.sets, "TFLOP/s"), (SMALL, 64, "GB/s")):
+        p = workloads.Problem("base-3 " + base.name, "ternary_b3", base.M, base.N, base.K, base.seed)
+        sets = make_sets(p, sets_n, torch, bw, distinct_weights=False)
+        steps = max(200, min(args.steps, 2000))
+        secs = time_launches(torch, bw, p, sets, steps, max(args.warmup, 3), dist)
+        t = max_over_ranks(torch, secs, dist) / steps
+        del sets
+        value = flops(p) / t / 1e12 if unit == "TFLOP/s" else algorithmic_bytes(p) / t / 1e9
+        out.append({"workload": p.name, "mode": p.mode, "M": p.M, "N": p.N, "K": p.K, "value": value, "unit": unit,
+                    "us_per_launch": t * 1e6, "packed_bytes": packed_weight_bytes(p.mode, p.N, p.K),
+                    "int2_packed_bytes": packed_weight_bytes("ternary", p.N, p.K),
+                    "plan": bw.gemm_plan(p.M, p.N, p.K, p.mode)})
+    return out
 
 
 def cublas_fp16_same_run(torch, n=8192, seconds=0.4):
