@@ -210,14 +210,14 @@ int smem_opt_in(int bytes) {
 }
 
 // Clusters of `ksplit` CTAs that can be resident at once (0 if unknown).
-template <int MODE, int BLOCK_T, int OCC>
+template <int MODE, int BLOCK_T>
 int resident_clusters(int ksplit) {
-  using T = GemmTile<MODE, BLOCK_T, OCC>;
+  using T = GemmTile<MODE, BLOCK_T>;
   static std::mutex mu;
   static int cache[9] = {0};
   std::lock_guard<std::mutex> lock(mu);
   if (ksplit < 1 || ksplit > 8) return 0;
-  if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T, OCC>>(T::kSmemBytes) != BONSAI_OK) return 0;
+  if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T>>(T::kSmemBytes) != BONSAI_OK) return 0;
   if (cache[ksplit] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, ksplit);
@@ -231,7 +231,7 @@ int resident_clusters(int ksplit) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, lowbit_gemm_kernel<MODE, BLOCK_T, OCC>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, lowbit_gemm_kernel<MODE, BLOCK_T>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       n = -1;
     }
@@ -240,12 +240,12 @@ int resident_clusters(int ksplit) {
   return cache[ksplit] > 0 ? cache[ksplit] : 0;
 }
 
-template <int MODE, int BLOCK_T, int OCC>
+template <int MODE, int BLOCK_T>
 int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, int ksplit,
                 uint16_t* out, cudaStream_t stream) {
-  using T = GemmTile<MODE, BLOCK_T, OCC>;
-  auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T, OCC>;
-  if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T, OCC>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
+  using T = GemmTile<MODE, BLOCK_T>;
+  auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T>;
+  if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
 
   CUtensorMap map_act, map_w, map_out;
   if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, BLOCK_T, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -393,7 +393,7 @@ void consider(int M, int N, int K, Plan* best) {
   // Base-3 ranges start on 4-group blocks: at most groups / 4 of them.
   const int max_ks = MODE == BONSAI_TERNARY_B3 ? (groups / kB3BlockGroups > 1 ? groups / kB3BlockGroups : 1) : groups;
   for (int ks = 1; ks <= 8 && ks <= max_ks; ++ks) {
-    const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T, 1>(ks);
+    const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T>(ks);
     if (per_wave <= 0) continue;
     const int waves = (tiles + per_wave - 1) / per_wave;
     const bool persistent = BLOCK_T == 256 && ks == 1 && use_persistent<MODE>(M, N, K);
@@ -439,11 +439,11 @@ int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales,
   const Plan p = plan_gemm<MODE>(M, N, K);
   if (p.persistent) return launch_gemm_persistent<MODE>(A, packed, scales, M, N, K, out, stream);
   switch (p.block_t) {
-    case 16: return launch_gemm<MODE, 16, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 32: return launch_gemm<MODE, 32, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 64: return launch_gemm<MODE, 64, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 128: return launch_gemm<MODE, 128, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 256: return launch_gemm<MODE, 256, 1>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 16: return launch_gemm<MODE, 16>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 32: return launch_gemm<MODE, 32>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 64: return launch_gemm<MODE, 64>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 128: return launch_gemm<MODE, 128>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 256: return launch_gemm<MODE, 256>(A, packed, scales, M, N, K, p.ksplit, out, stream);
     default: return BONSAI_ERR_CUDA;  // no plan: the occupancy queries failed
   }
 }

@@ -16,9 +16,10 @@
 //   TMEM ring  (warps 3-18, four per TMEM lane quadrant, taking groups in
 //                        turn) converters: each thread owns one weight row,
 //                        turns the group's words into exact FP16 products
-//                        (binary: sign bit over s; ternary: the shifted 2-bit
-//                        field is 2t, times s) and writes them to a TMEM
-//                        stage with tcgen05.st.
+//                        (binary: sign bit over s; ternary INT2: the shifted
+//                        2-bit field is 2t, times s; base-3: digits stepped
+//                        out of two bytes at a time, t, times s) and writes
+//                        them to a TMEM stage with tcgen05.st.
 //   warp 1               allocates TMEM; one thread issues
 //                        tcgen05.mma.kind::f16 (M=128, N=BLOCK_T, K=16) x 8
 //                        per group, A from TMEM, B from shared memory, FP32
@@ -60,11 +61,10 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
   return p;
 }
 
-// OCC = CTAs per SM.  OCC 1: a CTA owns all 512 TMEM columns and most of
-// shared memory.  OCC 2 (tiles of at most 128 tokens): two CTAs share an SM,
-// 256 TMEM columns and ~110 KB of shared memory each, so that one CTA's
-// prologue and epilogue overlap the other's MMAs.
-template <int MODE, int BLOCK_T, int OCC = 1>
+// One CTA per SM: a CTA owns all 512 TMEM columns and most of shared memory.
+// (Two CTAs per SM with 128-token tiles, 256 TMEM columns each, measured 15%
+// slower on the M=4608 workload.)
+template <int MODE, int BLOCK_T>
 struct GemmTile {
   static constexpr int kRows = 128;  // weight rows per tile (MMA M)
   static constexpr bool kB3 = MODE == BONSAI_TERNARY_B3;
@@ -75,8 +75,7 @@ struct GemmTile {
   // Activation stages: as many as fit next to the word ring and the scales,
   // so that narrow tiles keep a split-K CTA's whole K range in flight.
   static constexpr int kActStages =
-      OCC == 2 ? (64 * 1024) / kActStageBytes
-               : (BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : (96 * 1024) / kActStageBytes));
+      BLOCK_T >= 256 ? 3 : (BLOCK_T >= 128 ? 4 : (96 * 1024) / kActStageBytes);
   // A word stage is 128 bytes of every row: 4 ternary or 8 binary groups,
   // one TMA box with 128-byte swizzling.
   // Base-3: one 112-byte block (4 groups) of every row per stage, without
@@ -89,13 +88,13 @@ struct GemmTile {
   static constexpr int kGroupAlign = kB3 ? kB3BlockGroups : 1;
   // Small token tiles are bandwidth-bound: enough word stages to keep every
   // load of a split-K CTA in flight at once.
-  static constexpr int kWStages = (OCC == 2 || BLOCK_T >= 256) ? 2 : 4;
+  static constexpr int kWStages = BLOCK_T >= 256 ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
-  static constexpr int kScaleBytes = (OCC == 2 || BLOCK_T >= 256) ? 0 : 32768;
+  static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
   // Converter warps: 2 or 4 per TMEM lane quadrant.  (Five per quadrant on
   // narrow tiles measured 2-5% slower: their tensor-memory stores, not the
   // number of groups in conversion, set the pace.)
-  static constexpr int kConvWarps = OCC == 2 ? 8 : 16;
+  static constexpr int kConvWarps = 16;
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
   // Epilogue: the quadrant's warps split the token columns, 8 at least each:
   // the most warps (up to kWarpsPerQuad) that divide BLOCK_T / 8.
@@ -104,7 +103,7 @@ struct GemmTile {
   // two activation producers for tiles of up to 128 tokens, where one thread
   // issuing every MMA and polling every barrier is the serial limit.  A
   // 256-token accumulator fills half of TMEM, so those tiles keep one.
-  static constexpr int kMmaThreads = (OCC == 1 && BLOCK_T <= 128) ? 2 : 1;
+  static constexpr int kMmaThreads = BLOCK_T <= 128 ? 2 : 1;
   static constexpr int kActWarpB = 3 + kConvWarps;  // second activation producer
   static constexpr int kMmaWarpB = 4 + kConvWarps;  // second MMA issuer (idle when kMmaThreads == 1)
   static constexpr int kThreads = 32 * (5 + kConvWarps);
@@ -117,7 +116,7 @@ struct GemmTile {
   // after the accumulators.  A stage is reused only after the MMAs that read
   // it completed, so the number of stages is the number of groups in flight
   // between the converters and the tensor core.
-  static constexpr int kTmemCols = 512 / OCC;
+  static constexpr int kTmemCols = 512;
   static constexpr int kTStagesFit = (kTmemCols - kACol0) / 64;
   // With two MMA-issuing warps the stage count has the parity of
   // kWarpsPerQuad (one stage is left unused otherwise); see the assertion below.
@@ -130,14 +129,13 @@ struct GemmTile {
   static constexpr int kNumBars = 2 * kActStages + 2 * kTStages + 2 * kWStages + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemNeeded = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
-  // OCC 1: a second CTA could not get its 512 TMEM columns, so shared memory
-  // keeps it off the SM.
-  static constexpr int kSmemBytes = (OCC == 1 && kSmemNeeded < 116 * 1024) ? 116 * 1024 : kSmemNeeded;
+  // A second CTA could not get its 512 TMEM columns, so shared memory keeps
+  // it off the SM.
+  static constexpr int kSmemBytes = kSmemNeeded < 116 * 1024 ? 116 * 1024 : kSmemNeeded;
 
   static constexpr float kOutScale = MODE == BONSAI_TERNARY_INT2 ? 0.5f : 1.0f;  // INT2 converts to 2ts
   static_assert(BLOCK_T % 16 == 0 && BLOCK_T >= 16 && BLOCK_T <= 256, "MMA N for M=128");
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
-  static_assert(OCC == 1 || OCC == 2, "one or two CTAs per SM");
   static_assert(kACol0 + kTStages * 64 <= kTmemCols && kTStages >= 2, "TMEM budget");
   // Parity waits on a TMEM stage are unambiguous only if the converter is at
   // most one use ahead of the MMAs: when a converter waits for the MMAs of
@@ -149,7 +147,7 @@ struct GemmTile {
   static_assert(kWarpsPerQuad <= kTStages, "converter warps per quadrant <= TMEM stages");
   static_assert(kWGroups % kWarpsPerQuad == 0, "every converter warp reads every full word stage");
   static_assert(kMmaThreads == 1 || (kTStages - kWarpsPerQuad) % 2 == 0, "same MMA warp for groups i-q-TS, i-2TS");
-  static_assert(kSmemBytes <= (OCC == 1 ? 227 * 1024 : 113 * 1024), "shared memory per CTA");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(kActStages >= 2, "activation ring depth");
   static_assert(BLOCK_T * kRows * 2 <= kActStages * kActStageBytes, "output tile fits the act ring");
   static_assert(kRows * BLOCK_T * 4 <= kActStages * kActStageBytes, "partial fits the act ring");
@@ -254,12 +252,12 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
 };
 
-template <int MODE, int BLOCK_T, int OCC>
-__global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T, OCC>::kThreads, OCC)
+template <int MODE, int BLOCK_T>
+__global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_s,
                        const GemmArgs args) {
-  using T = GemmTile<MODE, BLOCK_T, OCC>;
+  using T = GemmTile<MODE, BLOCK_T>;
   constexpr int AS = T::kActStages, TS = T::kTStages, WS = T::kWStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
