@@ -477,9 +477,17 @@ int pipeline_for_device(HostPipeline** out) {
     for (int c = 0; ok && c < kMaxChunks; ++c)
       ok = cudaEventCreateWithFlags(&p.copied[c], ev) == cudaSuccess &&
            cudaEventCreateWithFlags(&p.computed[c], ev) == cudaSuccess;
-    if (!ok) {
+    if (!ok) {  // release what was created; the next call starts over
       cudaGetLastError();
-      return BONSAI_ERR_CUDA;  // partial objects are kept and retried next time
+      for (cudaStream_t* st : {&p.in, &p.comp, &p.out})
+        if (*st) cudaStreamDestroy(*st), *st = nullptr;
+      for (cudaEvent_t* ev : {&p.start, &p.done})
+        if (*ev) cudaEventDestroy(*ev), *ev = nullptr;
+      for (int c = 0; c < kMaxChunks; ++c) {
+        if (p.copied[c]) cudaEventDestroy(p.copied[c]), p.copied[c] = nullptr;
+        if (p.computed[c]) cudaEventDestroy(p.computed[c]), p.computed[c] = nullptr;
+      }
+      return BONSAI_ERR_CUDA;
     }
     p.ready = true;
   }
