@@ -221,7 +221,9 @@ def run_reference(args):
     d = workloads.make(p)
     packed = oracle.pack(d["codes"], p.mode)
     threads = oracle.default_threads()
-    rows, n_blk = 16, 128
+    # 128 token rows per step: the oracle converts each weight row it uses to
+    # double once per call, which 16 rows would leave dominating the step
+    rows, n_blk = 128, 128
     # size each step so that warm-up + timed steps end within ~2.5 minutes
     t0 = time.perf_counter()
     oracle.gemm(d["A"][:rows], packed[:n_blk], d["scales"][:n_blk], p.K, p.mode, threads=threads, want_acc=False)
