@@ -80,6 +80,14 @@ def _load():
             lib.oracle_gemm.restype = ctypes.c_int
             lib.oracle_gemm_entries.argtypes = [P, P, P, I64, I64, I64, ctypes.c_int, P, P, I64, P, P, P]
             lib.oracle_gemm_entries.restype = ctypes.c_int
+            lib.oracle_gemm_w16.argtypes = [P, P, I64, I64, I64, P, P, P, ctypes.c_int]
+            lib.oracle_gemm_w16.restype = ctypes.c_int
+            lib.oracle_hqq4_pack.argtypes = [P, I64, I64, P]
+            lib.oracle_hqq4_pack.restype = ctypes.c_int
+            lib.oracle_hqq4_unpack.argtypes = [P, I64, I64, P]
+            lib.oracle_hqq4_unpack.restype = ctypes.c_int
+            lib.oracle_hqq4_dequant.argtypes = [P, P, P, I64, I64, P]
+            lib.oracle_hqq4_dequant.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -206,6 +214,60 @@ def gemm_entries(A_bits, packed, scales, K: int, mode, ms, ns):
                                      ms.size, _ptr(out), _ptr(acc), _ptr(absacc))
     _check(rc, "oracle_gemm_entries")
     return out, acc, absacc
+
+
+def gemm_w16(A_bits, w_bits, threads: int | None = None):
+    """out = A * W^T for FP16 weights given as bit patterns [N,K]; returns
+    (out_bits, acc, absacc) like gemm()."""
+    a = _c(A_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    M, K = a.shape
+    N = w.shape[0]
+    assert w.shape[1] == K
+    out = np.zeros((M, N), np.uint16)
+    acc = np.zeros((M, N), np.float64)
+    absacc = np.zeros((M, N), np.float64)
+    rc = _load().oracle_gemm_w16(_ptr(a), _ptr(w), M, N, K, _ptr(out), _ptr(acc), _ptr(absacc),
+                                 threads or default_threads())
+    _check(rc, "oracle_gemm_w16")
+    return out, acc, absacc
+
+
+# ------------------------------------------- 4-bit group-affine weights --
+HQQ_GROUP = 64
+
+
+def hqq4_pack(q) -> np.ndarray:
+    """uint8 q [N,K] in 0..15 -> uint32 words [N, K/8] (bonsai_oracle.c)."""
+    c = _c(q, np.uint8)
+    N, K = c.shape
+    out = np.zeros((N, K // 8), np.uint32)
+    _check(_load().oracle_hqq4_pack(_ptr(c), N, K, _ptr(out)), "oracle_hqq4_pack")
+    return out
+
+
+def hqq4_unpack(packed, K: int) -> np.ndarray:
+    p = _c(packed, np.uint32)
+    out = np.zeros((p.shape[0], K), np.uint8)
+    _check(_load().oracle_hqq4_unpack(_ptr(p), p.shape[0], K, _ptr(out)), "oracle_hqq4_unpack")
+    return out
+
+
+def hqq4_dequant(packed, scales, zeros, K: int) -> np.ndarray:
+    """-> fp16 bits of w = fp16(fp16(q - z) * s), groups of 64 along K."""
+    p = _c(packed, np.uint32)
+    s = _c(scales, np.uint16)
+    z = _c(zeros, np.uint16)
+    N = p.shape[0]
+    out = np.zeros((N, K), np.uint16)
+    _check(_load().oracle_hqq4_dequant(_ptr(p), _ptr(s), _ptr(z), N, K, _ptr(out)), "oracle_hqq4_dequant")
+    return out
+
+
+def hqq4_gemm(A_bits, packed, scales, zeros, K: int, threads: int | None = None):
+    """out = A * W^T for 4-bit group-affine weights: the dequantised FP16
+    weights, then one double sum per output."""
+    return gemm_w16(A_bits, hqq4_dequant(packed, scales, zeros, K), threads)
 
 
 def ulp16(ref_bits) -> np.ndarray:

@@ -34,6 +34,16 @@
  * with its alignment padding; the pages' 1.71-bit figure is log2(3) +
  * 16/128, and INT2 storage spends 2 bits) is this project's own too; it is
  * defined at pack_b3_group.
+ *
+ * 4-bit group-affine weights.  The pages name "4-bit HQQ" for the text
+ * encoder ("Cómo Bonsai Ternary 4B revoluciona la difusión texto-imagen",
+ * section "Arquitectura de despliegue y eficiencia en tiempo de ejecución")
+ * and give nothing more.  This project reads it
+ * as HQQ's published scheme: an unsigned 4-bit q per weight, and per group of
+ * 64 weights along K an FP16 scale s and FP16 zero z, the weight being
+ * evaluated in FP16 as w = fp16(fp16(q - z) * s).  The group size, the zero
+ * as an FP16 value and the packing (oracle_hqq4_pack) are this reading's
+ * choices; none of it is pinned by the pages.
  */
 #include <math.h>
 #include <pthread.h>
@@ -376,6 +386,9 @@ static int weights_as_double(const uint32_t* packed, const uint16_t* scales, int
   return ORACLE_OK;
 }
 
+static int gemm_with_weights(const uint16_t* A, double* w, int64_t M, int64_t N, int64_t K, uint16_t* out,
+                             double* acc, double* absacc, int nthreads);
+
 /* out = A * W^T, one double accumulation per output.  Rows of the output are
  * split across nthreads worker threads (each output is still one sequential
  * sum, so the thread count does not change any result). */
@@ -385,10 +398,26 @@ int oracle_gemm(const uint16_t* A, const uint32_t* packed, const uint16_t* scale
   int rc = check_mode_shape(N, K, mode);
   if (rc != ORACLE_OK) return rc;
   if (M < 0) return ORACLE_ERR_SHAPE;
-  if (nthreads < 1) nthreads = 1;
   double* w = NULL;
   rc = weights_as_double(packed, scales, N, K, mode, &w);
   if (rc != ORACLE_OK) return rc;
+  return gemm_with_weights(A, w, M, N, K, out, acc, absacc, nthreads);
+}
+
+/* The same product for FP16 weights given directly, [N,K] row-major. */
+int oracle_gemm_w16(const uint16_t* A, const uint16_t* w16, int64_t M, int64_t N, int64_t K, uint16_t* out,
+                    double* acc, double* absacc, int nthreads) {
+  if (M < 0 || N < 0 || K < 0) return ORACLE_ERR_SHAPE;
+  double* w = (double*)malloc((size_t)(N * K > 0 ? N * K : 1) * sizeof(double));
+  if (!w) return ORACLE_ERR_NOMEM;
+  oracle_half_to_double_array(w16, N * K, w);
+  return gemm_with_weights(A, w, M, N, K, out, acc, absacc, nthreads);
+}
+
+/* Takes ownership of w. */
+static int gemm_with_weights(const uint16_t* A, double* w, int64_t M, int64_t N, int64_t K, uint16_t* out,
+                             double* acc, double* absacc, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
   double* a = (double*)malloc((size_t)(M * K > 0 ? M * K : 1) * sizeof(double));
   if (!a) {
     free(w);
@@ -463,5 +492,71 @@ int oracle_gemm_entries(const uint16_t* A, const uint32_t* packed, const uint16_
   }
   free(t);
   free(w16);
+  return rc;
+}
+
+/* ---------------------------------------------- 4-bit group-affine (HQQ) -- */
+
+#define HQQ_GROUP 64
+
+/* Packing (this project's): words run along K, 8 weights per word; weight i
+ * of word j (k = 8 j + i) is the nibble at bit 16 (i % 2) + 4 (i / 2), so
+ * weights 2p and 2p+1 sit at the same offset of the two 16-bit halves.  Rows
+ * of K/8 words, row-major [N, K/8].  q must be in 0..15. */
+static int hqq4_bit(int i) { return 16 * (i & 1) + 4 * (i >> 1); }
+
+static int hqq4_check(int64_t N, int64_t K) {
+  if (N < 0 || K < 0) return ORACLE_ERR_SHAPE;
+  if (K % GROUP != 0) return ORACLE_ERR_SHAPE; /* whole 128-weight tiles, two affine groups each */
+  return ORACLE_OK;
+}
+
+int oracle_hqq4_pack(const uint8_t* q, int64_t N, int64_t K, uint32_t* packed) {
+  int rc = hqq4_check(N, K);
+  if (rc != ORACLE_OK) return rc;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < K / 8; ++j) {
+      uint32_t word = 0;
+      for (int i = 0; i < 8; ++i) {
+        const uint8_t v = q[n * K + 8 * j + i];
+        if (v > 15) return ORACLE_ERR_BAD_CODE;
+        word |= (uint32_t)v << hqq4_bit(i);
+      }
+      packed[n * (K / 8) + j] = word;
+    }
+  return ORACLE_OK;
+}
+
+int oracle_hqq4_unpack(const uint32_t* packed, int64_t N, int64_t K, uint8_t* q) {
+  int rc = hqq4_check(N, K);
+  if (rc != ORACLE_OK) return rc;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < K / 8; ++j) {
+      const uint32_t word = packed[n * (K / 8) + j];
+      for (int i = 0; i < 8; ++i) q[n * K + 8 * j + i] = (uint8_t)((word >> hqq4_bit(i)) & 15u);
+    }
+  return ORACLE_OK;
+}
+
+/* w[n,k] = fp16(fp16(q - z) * s) with s = scales[n, k/64], z = zeros[n, k/64]:
+ * both steps are exact in double (a small integer minus an FP16 value; the
+ * product of two FP16 values) and rounded once each to FP16, which is the
+ * IEEE FP16 subtraction and multiplication. */
+int oracle_hqq4_dequant(const uint32_t* packed, const uint16_t* scales, const uint16_t* zeros, int64_t N,
+                        int64_t K, uint16_t* w) {
+  int rc = hqq4_check(N, K);
+  if (rc != ORACLE_OK) return rc;
+  uint8_t* q = (uint8_t*)malloc((size_t)(N * K > 0 ? N * K : 1));
+  if (!q) return ORACLE_ERR_NOMEM;
+  rc = oracle_hqq4_unpack(packed, N, K, q);
+  const int64_t groups = K / HQQ_GROUP;
+  for (int64_t n = 0; rc == ORACLE_OK && n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      const double s = oracle_half_to_double(scales[n * groups + k / HQQ_GROUP]);
+      const double z = oracle_half_to_double(zeros[n * groups + k / HQQ_GROUP]);
+      const uint16_t d = oracle_double_to_half((double)q[n * K + k] - z);
+      w[n * K + k] = oracle_double_to_half(oracle_half_to_double(d) * s);
+    }
+  free(q);
   return rc;
 }

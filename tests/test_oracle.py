@@ -513,3 +513,89 @@ def test_b3_weights_and_gemm_equal_int2_on_the_same_codes(oracle_mod):
     ms, ns = np.array([0, 8, 4]), np.array([32, 0, 17])
     e3 = oracle_mod.gemm_entries(d["A"], p3, d["scales"], 640, "ternary_b3", ms, ns)
     assert np.array_equal(e3[0], o2[ms, ns]) and np.array_equal(e3[1], a2[ms, ns])
+
+
+# ------------------------------------------- 4-bit group-affine weights --
+# The pages name "4-bit HQQ" for the text encoder and nothing more; the
+# oracle reads it as HQQ's scheme w = fp16(fp16(q - z) * s), groups of 64
+# along K, with this project's packing.  What is pinned below is that
+# reading's arithmetic and layout; the reading itself is unpinned.
+
+def test_hqq4_layout_shift_and_mask(oracle_mod):
+    """Weights 2p, 2p+1 of a word come out of (word >> 4p) & 0x000F000F as
+    the low and high 16-bit halves, for every nibble value in every slot."""
+    rng = np.random.default_rng(3)
+    q = rng.integers(0, 16, (64, 256)).astype(np.uint8)
+    q[0, :16] = np.arange(16)
+    words = oracle_mod.hqq4_pack(q).astype(np.uint64)
+    for p in range(4):
+        pair = (words >> np.uint64(4 * p)) & np.uint64(0x000F000F)
+        assert np.array_equal(pair & np.uint64(0xFFFF), q[:, 2 * p::8].astype(np.uint64))
+        assert np.array_equal(pair >> np.uint64(16), q[:, 2 * p + 1::8].astype(np.uint64))
+    assert np.array_equal(oracle_mod.hqq4_unpack(oracle_mod.hqq4_pack(q), 256), q)
+    bad = q.copy()
+    bad[5, 7] = 16
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.hqq4_pack(bad)
+
+
+def _f16(bits):
+    return np.asarray(bits, np.uint16).view(np.float16)
+
+
+def test_hqq4_dequant_matches_ieee_fp16_arithmetic(oracle_mod):
+    """w = fp16(fp16(q - z) * s) against numpy's float16 operations (each an
+    exactly computed result rounded once): every scale pattern with random q
+    and zero, and zeros / scales at the special values."""
+    rng = np.random.default_rng(11)
+    N, K = 1024, 128
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    scales = np.arange(N * 2, dtype=np.uint32).astype(np.uint16).reshape(N, 2)  # 2048 of the patterns
+    scales[:, 1] = rng.integers(0, 65536, N).astype(np.uint16)
+    zeros = rng.integers(0, 65536, (N, 2)).astype(np.uint16)
+    specials = np.array([0x0000, 0x8000, 0x3C00, 0x4700, 0x4B80, 0x7C00, 0xFC00, 0x7E00, 0x0001, 0x03FF],
+                        np.uint16)
+    zeros[:len(specials), 0] = specials
+    scales[len(specials):2 * len(specials), 0] = specials
+    got = oracle_mod.hqq4_dequant(oracle_mod.hqq4_pack(q), scales, zeros, K)
+    with np.errstate(all="ignore"):
+        zz = np.repeat(_f16(zeros), 64, axis=1)
+        ss = np.repeat(_f16(scales), 64, axis=1)
+        want = ((q.astype(np.float16) - zz).astype(np.float16) * ss).astype(np.float16)
+    assert np.all(nan_equal(got, want.view(np.uint16)))
+    for start in range(0, 65536, 8192):  # every scale pattern once, with q and z varying
+        s_all = (np.arange(start, start + 8192, dtype=np.uint32).astype(np.uint16)).reshape(-1, 2)
+        z_all = rng.integers(0, 65536, s_all.shape).astype(np.uint16)
+        q_all = rng.integers(0, 16, (s_all.shape[0], 128)).astype(np.uint8)
+        got = oracle_mod.hqq4_dequant(oracle_mod.hqq4_pack(q_all), s_all, z_all, 128)
+        with np.errstate(all="ignore"):
+            want = ((q_all.astype(np.float16) - np.repeat(_f16(z_all), 64, axis=1)).astype(np.float16) *
+                    np.repeat(_f16(s_all), 64, axis=1)).astype(np.float16)
+        assert np.all(nan_equal(got, want.view(np.uint16)))
+
+
+def nan_equal(a, b):
+    a = np.asarray(a, np.uint16)
+    b = np.asarray(b, np.uint16)
+    an, bn = np.isnan(a.view(np.float16)), np.isnan(b.view(np.float16))
+    return np.where(an | bn, an & bn, a == b)
+
+
+def test_hqq4_gemm_all_ones_closed_form(oracle_mod):
+    """With all-ones activations every output's double sum is exactly the sum
+    of the row's FP16 weights (each a multiple of 2^-24 below 2^16, so the
+    sums are exact in double)."""
+    rng = np.random.default_rng(13)
+    N, K = 40, 512
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    scales = np.float16(rng.uniform(0.001, 0.1, (N, K // 64))).view(np.uint16)
+    zeros = np.float16(rng.uniform(0.0, 15.0, (N, K // 64))).view(np.uint16)
+    packed = oracle_mod.hqq4_pack(q)
+    w = ((q.astype(np.float16) - np.repeat(_f16(zeros), 64, axis=1)).astype(np.float16) *
+         np.repeat(_f16(scales), 64, axis=1)).astype(np.float16)
+    want = w.astype(np.float64).sum(axis=1)
+    A = np.full((3, K), 0x3C00, np.uint16)  # 1.0
+    out, acc, absacc = oracle_mod.hqq4_gemm(A, packed, scales, zeros, K)
+    assert np.array_equal(acc, np.broadcast_to(want, acc.shape))
+    assert np.array_equal(absacc, np.broadcast_to(np.abs(w.astype(np.float64)).sum(axis=1), acc.shape))
+    assert np.array_equal(out, oracle_mod.double_to_half_bits(acc))

@@ -29,6 +29,14 @@ MUTATIONS = {
                                                 "if (k < GROUP) t[k] = (int8_t)(1 - q);"),
     "base-3 value stored rounded down": ("out[j] = (uint8_t)((256 * value + 242) / 243);",
                                          "out[j] = (uint8_t)((256 * value) / 243);"),
+    "4-bit halves swapped": ("static int hqq4_bit(int i) { return 16 * (i & 1) + 4 * (i >> 1); }",
+                             "static int hqq4_bit(int i) { return 16 * (1 - (i & 1)) + 4 * (i >> 1); }"),
+    "4-bit zero added": ("oracle_double_to_half((double)q[n * K + k] - z);",
+                         "oracle_double_to_half((double)q[n * K + k] + z);"),
+    "4-bit affine group of 128": ("#define HQQ_GROUP 64", "#define HQQ_GROUP 128"),
+    "4-bit difference not rounded to FP16": (
+        "w[n * K + k] = oracle_double_to_half(oracle_half_to_double(d) * s);",
+        "w[n * K + k] = oracle_double_to_half(((double)q[n * K + k] - z) * s + 0.0 * d);"),
     "base-3 groups packed without blocks": (
         "return g / B3_BLOCK_GROUPS * B3_BLOCK_BYTES + g % B3_BLOCK_GROUPS * B3_GROUP_BYTES;",
         "return g * B3_GROUP_BYTES;"),
