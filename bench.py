@@ -488,6 +488,42 @@ def time_formats(torch, bw, args, dist, peaks, peaks_kind):
                     "us_per_launch": t * 1e6, "packed_bytes": packed_weight_bytes(p.mode, p.N, p.K),
                     "int2_packed_bytes": packed_weight_bytes("ternary", p.N, p.K),
                     "plan": bw.gemm_plan(p.M, p.N, p.K, p.mode)})
+    # 4-bit group-affine weights (the text encoder's format) on the headline shape
+    p = WORKLOAD
+    d = workloads.make_hqq4(1, p.N, p.K, seed=p.seed)
+    packed = bw.hqq4_pack(torch.from_numpy(d["q"]).cuda())
+    s = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+    z = torch.from_numpy(d["zeros"].view(np.int16)).view(torch.float16).cuda()
+    rng = np.random.default_rng(p.seed)
+    sets = [(torch.from_numpy(workloads.activations(rng, p.M, p.K).view(np.int16)).view(torch.float16).cuda(),
+             packed.clone(), s.clone(), z.clone(), torch.empty((p.M, p.N), dtype=torch.float16, device="cuda"))
+            for _ in range(args.sets)]
+
+    def launch(i):
+        A, pk, sc, zc, o = sets[i % len(sets)]
+        bw.hqq4_gemm(A, pk, sc, zc, out=o)
+
+    for i in range(3):
+        launch(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(len(sets)):
+            launch(i)
+    steps = max(200, min(args.steps, 2000)) // len(sets) * len(sets)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps // len(sets)):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / steps
+    del graph, sets
+    out.append({"workload": "4-bit group-affine " + p.name, "mode": "hqq4", "M": p.M, "N": p.N, "K": p.K,
+                "value": flops(p) / t / 1e12, "unit": "TFLOP/s", "us_per_launch": t * 1e6,
+                "packed_bytes": p.N * p.K // 2, "plan": bw.gemm_plan(p.M, p.N, p.K, "hqq4")})
     return out
 
 

@@ -32,6 +32,10 @@ SIGNATURES = {
     "bonsai_pack": (ctypes.c_int, [_P, _I64, _I64, ctypes.c_int, _P, _P]),
     "bonsai_dequant": (ctypes.c_int, [_P, _P, _I64, _I64, ctypes.c_int, _P, _P]),
     "bonsai_lowbit_gemm": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P]),
+    "bonsai_hqq4_packed_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "bonsai_hqq4_pack": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "bonsai_hqq4_dequant": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
+    "bonsai_hqq4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "bonsai_lowbit_gemm_host": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P]),
     "bonsai_gemm_plan": (ctypes.c_int, [_I64, _I64, _I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
@@ -188,11 +192,52 @@ def lowbit_gemm_host(A_host: torch.Tensor, packed: torch.Tensor, scales: torch.T
     return out_host
 
 
+# ------------------------------------------- 4-bit group-affine weights --
+HQQ4 = 4  # mode value for gemm_plan
+HQQ_GROUP = 64
+
+
+def hqq4_pack(q: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """uint8 q [N,K] (0..15) on the device -> packed words (int32 view) [N, K/8]."""
+    N, K = q.shape
+    if out is None:
+        out = torch.empty((N, K // 8), dtype=torch.int32, device=q.device)
+    _check(lib().bonsai_hqq4_pack(_dev(q, "q", torch.uint8), N, K, _dev(out, "out", torch.int32), _stream()),
+           "bonsai_hqq4_pack")
+    return out
+
+
+def hqq4_dequant(packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, K: int,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """-> FP16 [N,K] with w = fp16(fp16(q - z) * s), groups of 64 along K."""
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    _check(lib().bonsai_hqq4_dequant(_dev(packed, "packed"), _dev(scales, "scales", torch.float16),
+                                     _dev(zeros, "zeros", torch.float16), N, K, _dev(out, "out", torch.float16),
+                                     _stream()), "bonsai_hqq4_dequant")
+    return out
+
+
+def hqq4_gemm(A: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+              out: torch.Tensor | None = None) -> torch.Tensor:
+    """out[M,N] = A[M,K] * W^T with 4-bit group-affine weights."""
+    M, K = A.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib().bonsai_hqq4_gemm(_dev(A, "A", torch.float16), _dev(packed, "packed"),
+                                  _dev(scales, "scales", torch.float16), _dev(zeros, "zeros", torch.float16),
+                                  M, N, K, _dev(out, "out", torch.float16), _stream()), "bonsai_hqq4_gemm")
+    return out
+
+
 def gemm_plan(M: int, N: int, K: int, mode) -> dict:
     """The launch bonsai_lowbit_gemm makes: tokens per tile, K split, CTAs,
     output tiles (fewer CTAs than tiles x split: the persistent form)."""
     bt, ks, ctas, tiles = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    _check(lib().bonsai_gemm_plan(M, N, K, _mode(mode), ctypes.byref(bt), ctypes.byref(ks), ctypes.byref(ctas),
+    m = HQQ4 if mode in (HQQ4, "hqq4") else _mode(mode)
+    _check(lib().bonsai_gemm_plan(M, N, K, m, ctypes.byref(bt), ctypes.byref(ks), ctypes.byref(ctas),
                                   ctypes.byref(tiles)), "bonsai_gemm_plan")
     return {"block_t": bt.value, "ksplit": ks.value, "ctas": ctas.value, "tiles": tiles.value}
 

@@ -27,6 +27,7 @@ bool valid_mode(int mode) {
 // Packed words of one row: K/32 (binary), K/16 (INT2), 28 per 4 groups (base-3).
 int64_t row_words(int64_t K, int mode) {
   if (mode == BONSAI_TERNARY_B3) return (K / kGroup + kB3BlockGroups - 1) / kB3BlockGroups * (kB3BlockBytes / 4);
+  if (mode == kModeHqq4) return K / 8;
   return K / (mode == BONSAI_BINARY ? 32 : 16);
 }
 
@@ -241,7 +242,8 @@ int resident_clusters(int ksplit) {
 }
 
 template <int MODE, int BLOCK_T>
-int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, int ksplit,
+int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, const uint16_t* zeros, int M, int N,
+                int K, int ksplit,
                 uint16_t* out, cudaStream_t stream) {
   using T = GemmTile<MODE, BLOCK_T>;
   auto kernel = lowbit_gemm_kernel<MODE, BLOCK_T>;
@@ -280,6 +282,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
 
   GemmArgs args;
   args.scales = scales;
+  args.zeros = zeros;
   args.out = out;
   args.M = M;
   args.N = N;
@@ -318,13 +321,17 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, i
 template <int MODE>
 bool use_persistent(int M, int N, int K) {
   using T = PersistTile<MODE>;
-  if (M <= 128 || K % (kGroup * T::kWGroups) != 0) return false;
+  // Whole word stages per tile, and a group count per tile that is a
+  // multiple of 4 (each converter warp keeps its TMEM stage across tiles).
+  const int per_stage = T::kWGroups > 4 ? T::kWGroups : 4;
+  if (M <= 128 || K % (kGroup * per_stage) != 0) return false;
   const int64_t tiles = static_cast<int64_t>((N + T::kRows - 1) / T::kRows) * ((M + T::kBlockT - 1) / T::kBlockT);
   return tiles > sm_count();
 }
 
 template <int MODE>
-int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
+int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t* scales, const uint16_t* zeros, int M,
+                           int N, int K,
                            uint16_t* out, cudaStream_t stream) {
   using T = PersistTile<MODE>;
   auto kernel = lowbit_gemm_persistent_kernel<MODE>;
@@ -335,6 +342,7 @@ int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t
   if (!make_weight_map(&map_w, packed, N, K, MODE)) return BONSAI_ERR_CUDA;
   PersistArgs args;
   args.scales = scales;
+  args.zeros = zeros;
   args.out = out;
   args.M = M;
   args.N = N;
@@ -434,16 +442,17 @@ Plan plan_gemm(int M, int N, int K) {
 }
 
 template <int MODE>
-int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K,
+int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, const uint16_t* zeros, int M, int N,
+                  int K,
                   uint16_t* out, cudaStream_t stream) {
   const Plan p = plan_gemm<MODE>(M, N, K);
-  if (p.persistent) return launch_gemm_persistent<MODE>(A, packed, scales, M, N, K, out, stream);
+  if (p.persistent) return launch_gemm_persistent<MODE>(A, packed, scales, zeros, M, N, K, out, stream);
   switch (p.block_t) {
-    case 16: return launch_gemm<MODE, 16>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 32: return launch_gemm<MODE, 32>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 64: return launch_gemm<MODE, 64>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 128: return launch_gemm<MODE, 128>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-    case 256: return launch_gemm<MODE, 256>(A, packed, scales, M, N, K, p.ksplit, out, stream);
+    case 16: return launch_gemm<MODE, 16>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+    case 32: return launch_gemm<MODE, 32>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+    case 64: return launch_gemm<MODE, 64>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+    case 128: return launch_gemm<MODE, 128>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+    case 256: return launch_gemm<MODE, 256>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     default: return BONSAI_ERR_CUDA;  // no plan: the occupancy queries failed
   }
 }
@@ -527,7 +536,7 @@ int gemm_host_pipelined(const uint16_t* A_host, const void* packed, const uint16
                         p->in) != cudaSuccess ||
         cudaEventRecord(p->copied[c], p->in) != cudaSuccess || cudaStreamWaitEvent(p->comp, p->copied[c], 0) != cudaSuccess)
       return BONSAI_ERR_CUDA;
-    rc = dispatch_gemm<MODE>(A_dev + a_off, packed, scales, static_cast<int>(m), static_cast<int>(N),
+    rc = dispatch_gemm<MODE>(A_dev + a_off, packed, scales, nullptr, static_cast<int>(m), static_cast<int>(N),
                              static_cast<int>(K), out_dev + o_off, p->comp);
     if (rc != BONSAI_OK) return rc;
     if (cudaEventRecord(p->computed[c], p->comp) != cudaSuccess ||
@@ -631,9 +640,10 @@ int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* sc
   if (!A || !packed || !scales) return BONSAI_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(packed) || !aligned16(scales)) return BONSAI_ERR_ALIGN;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-  if (mode == BONSAI_BINARY) return dispatch_gemm<BONSAI_BINARY>(A, packed, scales, m, n, k, out, st);
-  if (mode == BONSAI_TERNARY_B3) return dispatch_gemm<BONSAI_TERNARY_B3>(A, packed, scales, m, n, k, out, st);
-  return dispatch_gemm<BONSAI_TERNARY_INT2>(A, packed, scales, m, n, k, out, st);
+  if (mode == BONSAI_BINARY) return dispatch_gemm<BONSAI_BINARY>(A, packed, scales, nullptr, m, n, k, out, st);
+  if (mode == BONSAI_TERNARY_B3)
+    return dispatch_gemm<BONSAI_TERNARY_B3>(A, packed, scales, nullptr, m, n, k, out, st);
+  return dispatch_gemm<BONSAI_TERNARY_INT2>(A, packed, scales, nullptr, m, n, k, out, st);
 }
 
 int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
@@ -660,8 +670,65 @@ int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const ui
   return gemm_host_pipelined<BONSAI_TERNARY_INT2>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
 }
 
+// ------------------------------------------ 4-bit group-affine weights --
+size_t bonsai_hqq4_packed_bytes(int64_t N, int64_t K) {
+  if (check_shape(0, N, K) != BONSAI_OK) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) / 2;
+}
+
+int bonsai_hqq4_pack(const uint8_t* q, int64_t N, int64_t K, void* packed, void* stream) {
+  int rc = check_shape(0, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (N == 0 || K == 0) return BONSAI_OK;
+  if (!q || !packed) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(packed)) return BONSAI_ERR_ALIGN;
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_pack_bad_code, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return BONSAI_ERR_CUDA;
+  const int64_t words = N * K / 8;
+  pack_hqq4_kernel<<<grid_for(words / 4, 256), 256, 0, st>>>(q, static_cast<uint32_t*>(packed), words);
+  if ((rc = launch_status()) != BONSAI_OK) return rc;
+  unsigned bad = 0;
+  if (cudaMemcpyFromSymbolAsync(&bad, g_pack_bad_code, sizeof(bad), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return BONSAI_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BONSAI_ERR_CUDA;
+  return bad ? BONSAI_ERR_BAD_CODE : BONSAI_OK;
+}
+
+int bonsai_hqq4_dequant(const void* packed, const uint16_t* scales, const uint16_t* zeros, int64_t N, int64_t K,
+                        uint16_t* w, void* stream) {
+  int rc = check_shape(0, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (N == 0 || K == 0) return BONSAI_OK;
+  if (!packed || !scales || !zeros || !w) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(scales) || !aligned16(zeros) || !aligned16(w)) return BONSAI_ERR_ALIGN;
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dequant_hqq4_kernel<<<grid_for(N * K / 8, 256), 256, 0, st>>>(static_cast<const uint32_t*>(packed), scales, zeros,
+                                                                  w, N, K);
+  return launch_status();
+}
+
+int bonsai_hqq4_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, const uint16_t* zeros, int64_t M,
+                     int64_t N, int64_t K, uint16_t* out, void* stream) {
+  int rc = check_shape(M, N, K);
+  if (rc != BONSAI_OK) return rc;
+  if (M == 0 || N == 0) return BONSAI_OK;
+  if (!out || (K > 0 && (!A || !packed || !scales || !zeros))) return BONSAI_ERR_INVALID_ARG;
+  if (!aligned16(out) || (K > 0 && (!aligned16(A) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros))))
+    return BONSAI_ERR_ALIGN;
+  if ((rc = check_device()) != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 0)
+    return cudaMemsetAsync(out, 0, static_cast<size_t>(M) * N * 2, st) == cudaSuccess ? BONSAI_OK : BONSAI_ERR_CUDA;
+  return dispatch_gemm<kModeHqq4>(A, packed, scales, zeros, static_cast<int>(M), static_cast<int>(N),
+                                  static_cast<int>(K), out, st);
+}
+
 int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas, int* tiles) {
-  if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
+  if (!valid_mode(mode) && mode != kModeHqq4) return BONSAI_ERR_INVALID_ARG;
   int rc = check_shape(M, N, K);
   if (rc != BONSAI_OK) return rc;
   if (!block_t || !ksplit || !ctas || !tiles) return BONSAI_ERR_INVALID_ARG;
@@ -676,6 +743,7 @@ int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, in
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   const Plan p = mode == BONSAI_BINARY      ? plan_gemm<BONSAI_BINARY>(m, n, k)
                  : mode == BONSAI_TERNARY_B3 ? plan_gemm<BONSAI_TERNARY_B3>(m, n, k)
+                 : mode == kModeHqq4         ? plan_gemm<kModeHqq4>(m, n, k)
                                              : plan_gemm<BONSAI_TERNARY_INT2>(m, n, k);
   if (p.block_t == 0) return BONSAI_ERR_CUDA;
   *block_t = p.block_t;

@@ -36,8 +36,9 @@ struct PersistTile {
   static constexpr int kBlockT = 256;  // tokens per tile (MMA N)
   static constexpr int kRows = 128;    // weight rows per tile (MMA M)
   static constexpr bool kB3 = MODE == BONSAI_TERNARY_B3;
-  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : 8);  // held per group
-  static constexpr int kWGroups = kB3 ? kB3BlockGroups : 32 / kWordsPerGroup;    // groups per word stage
+  static constexpr bool kHqq = MODE == kModeHqq4;
+  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : (kHqq ? 16 : 8));  // held per group
+  static constexpr int kWGroups = kB3 ? kB3BlockGroups : 32 / kWordsPerGroup;  // groups per word stage
   static constexpr int kWRowBytes = kB3 ? kB3BlockBytes : 128;                  // bytes of a row per stage
   static constexpr int kSliceBytes = kBlockT * 128;     // 256 rows x 64 FP16
   static constexpr int kActStageBytes = 2 * kSliceBytes;
@@ -64,12 +65,16 @@ struct PersistTile {
   // stage `turn`, and its first group of a tile reuses the stage of the
   // previous tile's group ng - 4 + turn.
   static_assert(kTStages == 4 && kWarpsPerQuad == 4, "stage ownership by turn");
+  // Converter warps reading each word stage: all 16, or (4-bit weights, 2
+  // groups per stage) the 4 warps of each of its groups.
+  static constexpr int kWReaders = 4 * (kWGroups < kWarpsPerQuad ? kWGroups : kWarpsPerQuad);
   static_assert(kEpiCols % 16 == 0, "read-out in 16-column batches");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 struct PersistArgs {
   const uint16_t* scales;
+  const uint16_t* zeros;  // 4-bit group-affine weights only
   uint16_t* out;
   int M, N, K;
   int tiles_n;  // 128-row tiles along N; tile tau covers rows (tau % tiles_n) and tokens (tau / tiles_n)
@@ -121,7 +126,7 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
     }
     for (int s = 0; s < WS; ++s) {
       mbar_init(w_full0 + 8 * s, 1);
-      mbar_init(w_empty0 + 8 * s, T::kConvWarps);
+      mbar_init(w_empty0 + 8 * s, T::kWReaders);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, T::kConvWarps);
@@ -242,14 +247,25 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
     const bool convert_first = turn < TS - 1;
     bool ok = true;
 
+    // The group's scale (4-bit weights: its two scales, and the two zeros).
     auto scale_of = [&](int it, int i) -> uint32_t {
       const int n = tile_n0(it) + row;
-      return (it < ntiles && n < args.N) ? static_cast<uint32_t>(__ldg(args.scales + static_cast<size_t>(n) * groups + i))
-                                         : 0u;
+      if (it >= ntiles || n >= args.N) return 0u;
+      if constexpr (T::kHqq)
+        return __ldg(reinterpret_cast<const uint32_t*>(args.scales) + static_cast<size_t>(n) * groups + i);
+      return static_cast<uint32_t>(__ldg(args.scales + static_cast<size_t>(n) * groups + i));
+    };
+    auto zero_of = [&](int it, int i) -> uint32_t {
+      if constexpr (T::kHqq) {
+        const int n = tile_n0(it) + row;
+        if (it >= ntiles || n >= args.N) return 0u;
+        return __ldg(reinterpret_cast<const uint32_t*>(args.zeros) + static_cast<size_t>(n) * groups + i);
+      }
+      return 0u;
     };
 
     // Convert group i of tile it (running index c) into TMEM stage `turn`.
-    auto convert = [&](int it, int i, uint32_t sc) -> bool {
+    auto convert = [&](int it, int i, uint32_t sc, uint32_t zc) -> bool {
       const int c = it * groups + i;
       const int wc = it * nw + i / T::kWGroups;
       const int sw = wc % WS;
@@ -261,6 +277,15 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
       uint32_t words[T::kWordsPerGroup];
       if constexpr (T::kB3) {
         b3_group_words(reinterpret_cast<const uint32_t*>(wrow), pos, words);
+      } else if constexpr (T::kHqq) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16 * ((4 * pos + q4) ^ (row & 7)));
+          words[4 * q4] = q.x;
+          words[4 * q4 + 1] = q.y;
+          words[4 * q4 + 2] = q.z;
+          words[4 * q4 + 3] = q.w;
+        }
       } else if (MODE == BONSAI_BINARY) {
         const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16 * (pos ^ (row & 7)));
         words[0] = q.x;
@@ -280,10 +305,13 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
         words[7] = q1.w;
       }
       __syncwarp();
-      // Each warp reads kWGroups / 4 groups of a word stage; release after the last.
+      // Each reader has kWGroups / 4 groups of a word stage (or one, when a
+      // stage holds fewer groups than a quadrant has warps); release after the last.
       if (lane == 0 && pos + T::kWarpsPerQuad >= T::kWGroups) mbar_arrive(w_empty0 + 8 * sw);
       if constexpr (T::kB3)
         convert_group_b3(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + turn * 64);
+      else if constexpr (T::kHqq)
+        convert_group_hqq4(words, sc, zc, tmem + lane_base + T::kACol0 + turn * 64);
       else
         convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + turn * 64);
       tmem_store_wait();
@@ -331,14 +359,16 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
       return true;
     };
 
-    uint32_t sc_next = scale_of(0, turn);
+    uint32_t sc_next = scale_of(0, turn), zc_next = zero_of(0, turn);
     for (int it = 0; ok && it < ntiles; ++it) {
       for (int i = turn; i < groups; i += T::kWarpsPerQuad) {
-        const uint32_t sc = sc_next;
-        sc_next = i + T::kWarpsPerQuad < groups ? scale_of(it, i + T::kWarpsPerQuad) : scale_of(it + 1, turn);
+        const uint32_t sc = sc_next, zc = zc_next;
+        const bool last_of_tile = i + T::kWarpsPerQuad >= groups;
+        sc_next = last_of_tile ? scale_of(it + 1, turn) : scale_of(it, i + T::kWarpsPerQuad);
+        zc_next = last_of_tile ? zero_of(it + 1, turn) : zero_of(it, i + T::kWarpsPerQuad);
         const bool first_of_tile = i == turn && it > 0;
         if (first_of_tile && !convert_first && !(ok = read_out(it - 1))) break;
-        if (!(ok = convert(it, i, sc))) break;
+        if (!(ok = convert(it, i, sc, zc))) break;
         if (first_of_tile && convert_first && !(ok = read_out(it - 1))) break;
       }
     }

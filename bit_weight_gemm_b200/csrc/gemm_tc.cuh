@@ -69,7 +69,8 @@ struct GemmTile {
   static constexpr int kRows = 128;  // weight rows per tile (MMA M)
   static constexpr bool kB3 = MODE == BONSAI_TERNARY_B3;
   // Words a converter holds per group: 4 binary, 8 INT2, 7 base-3 (26 bytes).
-  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : 8);
+  static constexpr bool kHqq = MODE == kModeHqq4;
+  static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : (kHqq ? 16 : 8));
   static constexpr int kSliceBytes = BLOCK_T * 128;       // BLOCK_T rows x 64 FP16
   static constexpr int kActStageBytes = 2 * kSliceBytes;  // 128 K per stage
   // Activation stages: as many as fit next to the word ring and the scales,
@@ -90,7 +91,8 @@ struct GemmTile {
   // load of a split-K CTA in flight at once.
   static constexpr int kWStages = BLOCK_T >= 256 ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
-  static constexpr int kScaleBytes = BLOCK_T >= 256 ? 0 : 32768;
+  // (4-bit group-affine weights keep scale and zero pairs in registers.)
+  static constexpr int kScaleBytes = (BLOCK_T >= 256 || kHqq) ? 0 : 32768;
   // Converter warps: 2 or 4 per TMEM lane quadrant.  (Five per quadrant on
   // narrow tiles measured 2-5% slower: their tensor-memory stores, not the
   // number of groups in conversion, set the pace.)
@@ -145,7 +147,10 @@ struct GemmTile {
   // taking alternate groups, if both groups were issued by the same warp
   // (whose commit covers all its earlier MMAs): TS - kWarpsPerQuad even.
   static_assert(kWarpsPerQuad <= kTStages, "converter warps per quadrant <= TMEM stages");
-  static_assert(kWGroups % kWarpsPerQuad == 0, "every converter warp reads every full word stage");
+  // Converter warps reading each full word stage: every one of them, or (4-bit
+  // weights: 2 groups per stage) the four warps of each of its groups.
+  static constexpr int kWReaders = 4 * (kWGroups < kWarpsPerQuad ? kWGroups : kWarpsPerQuad);
+  static_assert(kWGroups % kWarpsPerQuad == 0 || kWarpsPerQuad % kWGroups == 0, "whole groups of readers");
   static_assert(kMmaThreads == 1 || (kTStages - kWarpsPerQuad) % 2 == 0, "same MMA warp for groups i-q-TS, i-2TS");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(kActStages >= 2, "activation ring depth");
@@ -202,7 +207,26 @@ __device__ __forceinline__ void convert_group_b3(const uint32_t* words, uint32_t
 template <int MODE>
 __device__ __forceinline__ int word_stage_x(int g0) {
   if (MODE == BONSAI_TERNARY_B3) return g0 / kB3BlockGroups * (kB3BlockBytes / 4);
-  return g0 * (MODE == BONSAI_BINARY ? 4 : 8);
+  return g0 * (MODE == BONSAI_BINARY ? 4 : (MODE == kModeHqq4 ? 16 : 8));
+}
+
+// 4-bit group-affine: the group's 16 words (K 0..63 in words 0-7 with the
+// first scale and zero, 64..127 in words 8-15 with the second) -> 64 TMEM
+// columns of FP16 pairs fp16(fp16(q - z) * s); column 4 j + p holds weights
+// 2p, 2p+1 of word j.  s_pair / z_pair hold the two groups' values.
+__device__ __forceinline__ void convert_group_hqq4(const uint32_t* words, uint32_t s_pair, uint32_t z_pair,
+                                                   uint32_t taddr) {
+  const uint32_t s_lo = __byte_perm(s_pair, 0u, 0x1010u), s_hi = __byte_perm(s_pair, 0u, 0x3232u);
+  const uint32_t z_lo = __byte_perm(z_pair, 0u, 0x1010u), z_hi = __byte_perm(z_pair, 0u, 0x3232u);
+  uint32_t v[8];
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int c = 4 * j + p;
+      v[c & 7] = hqq4_w_pair(hqq4_q_pair(words[j], p), j < 8 ? z_lo : z_hi, j < 8 ? s_lo : s_hi);
+      if ((c & 7) == 7) tmem_store_8(taddr + (c - 7), v);
+    }
 }
 
 // Boundary z of a split of `groups` into `ks` ranges, on multiples of ALIGN
@@ -244,6 +268,7 @@ __device__ __forceinline__ void sum_accumulators(uint32_t taddr, int used, float
 
 struct GemmArgs {
   const uint16_t* scales;
+  const uint16_t* zeros;  // 4-bit group-affine weights only
   uint16_t* out;
   int M, N, K;
   int ksplit;     // CTAs along K sharing one tile (the cluster size along z)
@@ -300,7 +325,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     }
     for (int s = 0; s < WS; ++s) {
       mbar_init(w_full0 + 8 * s, 1);
-      mbar_init(w_empty0 + 8 * s, T::kConvWarps);  // every converter warp reads each full stage
+      mbar_init(w_empty0 + 8 * s, T::kWReaders);  // the converter warps that read each full stage
     }
     mbar_init(dfull, T::kMmaThreads);
     mbar_init(s_full, 1);
@@ -458,23 +483,42 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       }
       named_barrier_sync(2, 32 * T::kConvWarps);
     }
-    uint32_t sq0 = 0, sq1 = 0;
+    uint32_t sq0 = 0, sq1 = 0, zq0 = 0, zq1 = 0;
     bool ok = !by_tma || warp_wait(s_full, 0, abort_flag, limit);
     constexpr int kStep = T::kWarpsPerQuad;
+    // Scale (4-bit weights: the group's two scales, and two zeros) of group i.
+    const uint32_t* srow2 =
+        T::kHqq ? reinterpret_cast<const uint32_t*>(args.scales) + static_cast<size_t>(n) * groups + g_begin : nullptr;
+    const uint32_t* zrow2 =
+        T::kHqq ? reinterpret_cast<const uint32_t*>(args.zeros) + static_cast<size_t>(n) * groups + g_begin : nullptr;
+    auto scale_at = [&](int i) -> uint32_t {
+      if (!row_ok || i >= ng) return 0u;
+      if constexpr (T::kHqq) return __ldg(srow2 + i);
+      return __ldg(srow + i);
+    };
+    auto zero_at = [&](int i) -> uint32_t {
+      if constexpr (T::kHqq) return (row_ok && i < ng) ? __ldg(zrow2 + i) : 0u;
+      return 0u;
+    };
     if (!staged) {
-      sq0 = (row_ok && turn < ng) ? __ldg(srow + turn) : 0u;
-      sq1 = (row_ok && turn + kStep < ng) ? __ldg(srow + turn + kStep) : 0u;
+      sq0 = scale_at(turn);
+      sq1 = scale_at(turn + kStep);
+      zq0 = zero_at(turn);
+      zq1 = zero_at(turn + kStep);
     }
     for (int i = turn; ok && i < ng; i += kStep) {
       const int wj = i / T::kWGroups;  // word stage of this group
       const int sw = wj % WS, st = i % TS;
-      uint32_t sc;
+      uint32_t sc, zc = 0;
       if (staged) {
         sc = sstage[row * s_stride + s_first + i];
       } else {
         sc = sq0;
         sq0 = sq1;
-        sq1 = (row_ok && i + 2 * kStep < ng) ? __ldg(srow + i + 2 * kStep) : 0u;
+        sq1 = scale_at(i + 2 * kStep);
+        zc = zq0;
+        zq0 = zq1;
+        zq1 = zero_at(i + 2 * kStep);
       }
       ok = warp_wait(w_full0 + 8 * sw, (wj / WS) & 1, abort_flag, limit) &&
            warp_wait(t_free0 + 8 * st, ((i / TS) & 1) ^ 1, abort_flag, limit);
@@ -487,6 +531,15 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       uint32_t words[T::kWordsPerGroup];
       if constexpr (T::kB3) {
         b3_group_words(reinterpret_cast<const uint32_t*>(wrow), pos, words);
+      } else if constexpr (T::kHqq) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16 * ((4 * pos + c) ^ (row & 7)));
+          words[4 * c] = q.x;
+          words[4 * c + 1] = q.y;
+          words[4 * c + 2] = q.z;
+          words[4 * c + 3] = q.w;
+        }
       } else if (MODE == BONSAI_BINARY) {
         const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16 * (pos ^ (row & 7)));
         words[0] = q.x;
@@ -506,14 +559,16 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
         words[7] = q1.w;
       }
       __syncwarp();
-      // Release the word stage after this warp's last group in it.  Every
-      // converter warp has a group in every full stage (kWGroups is a multiple
-      // of kWarpsPerQuad); only the CTA's last stage, which is never refilled,
-      // may lack some warps' arrivals.
+      // Release the word stage after this warp's last group in it.  The
+      // stage's readers (kWReaders) each have a group in every full stage;
+      // only the CTA's last stage, which is never refilled, may lack some
+      // readers' arrivals.
       const int stage_end = (wj + 1) * T::kWGroups < ng ? (wj + 1) * T::kWGroups : ng;
       if (lane == 0 && i + kStep >= stage_end) mbar_arrive(w_empty0 + 8 * sw);
       if constexpr (T::kB3)
         convert_group_b3(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
+      else if constexpr (T::kHqq)
+        convert_group_hqq4(words, sc, zc, tmem + lane_base + T::kACol0 + st * 64);
       else
         convert_group<MODE>(words, sc | (sc << 16), tmem + lane_base + T::kACol0 + st * 64);
       tmem_store_wait();

@@ -122,6 +122,79 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
   }
 }
 
+// ------------------------------------ 4-bit group-affine weights (HQQ) --
+// (bonsai.h.)  q in 0..15, 8 per word: weight i of a word at bit 16 (i%2) +
+// 4 (i/2), so (word >> 4p) & 0x000F000F holds weights 2p and 2p+1 in the
+// two halves; FP16 scale s and zero z per 64 weights along K;
+// w = fp16(fp16(q - z) * s).
+constexpr int kModeHqq4 = 4;  // kernel template mode of this format
+constexpr int kHqqGroup = 64;
+constexpr uint32_t kF16x2_1024 = 0x64006400u;
+
+// Weights 2p, 2p+1 of a word as the exact FP16 pair (q0, q1): the nibbles
+// under FP16's exponent of 1024, minus 1024.
+__device__ __forceinline__ uint32_t hqq4_q_pair(uint32_t word, int p) {
+  const uint32_t magic = ((word >> (4 * p)) & 0x000F000Fu) | kF16x2_1024;  // (1024 + q0, 1024 + q1)
+  uint32_t q;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q) : "r"(magic), "r"(kF16x2_1024));
+  return q;
+}
+
+// fp16(fp16(q - z) * s) for a pair, with z2 / s2 the group's zero / scale in
+// both halves: two IEEE FP16 operations, as the format defines.
+__device__ __forceinline__ uint32_t hqq4_w_pair(uint32_t q2, uint32_t z2, uint32_t s2) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(q2), "r"(z2));
+  return hmul2_bits(d, s2);
+}
+
+// Each thread packs 4 words (32 values, two 16-byte loads, one 16-byte store).
+__global__ void __launch_bounds__(256) pack_hqq4_kernel(const uint8_t* __restrict__ q, uint32_t* __restrict__ packed,
+                                                        int64_t total_words) {
+  const int64_t quads = total_words / 4;
+  bool ok = true;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < quads; t += (int64_t)gridDim.x * blockDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(q + t * 32);
+    const uint4 a = __ldg(src), b = __ldg(src + 1);
+    const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t value = (v[2 * j + (i >> 2)] >> (8 * (i & 3))) & 0xFFu;
+        ok &= value <= 15u;
+        word |= (value & 15u) << (16 * (i & 1) + 4 * (i >> 1));
+      }
+      w[j] = word;
+    }
+    reinterpret_cast<uint4*>(packed)[t] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (!__all_sync(0xffffffffu, ok) && lane_id() == 0) atomicOr(&g_pack_bad_code, 1u);
+}
+
+// Exact dequantisation: one thread per word (8 weights, one 16-byte store).
+__global__ void __launch_bounds__(256) dequant_hqq4_kernel(const uint32_t* __restrict__ packed,
+                                                           const uint16_t* __restrict__ scales,
+                                                           const uint16_t* __restrict__ zeros,
+                                                           uint16_t* __restrict__ w, int64_t N, int64_t K) {
+  const int64_t words_per_row = K / 8, groups = K / kHqqGroup;
+  const int64_t total = N * words_per_row;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = idx / words_per_row, j = idx - n * words_per_row;
+    const uint32_t word = __ldg(packed + idx);
+    const int64_t g = n * groups + (8 * j) / kHqqGroup;
+    const uint32_t s = __ldg(scales + g), z = __ldg(zeros + g);
+    const uint32_t s2 = s | (s << 16), z2 = z | (z << 16);
+    uint32_t v[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) v[p] = hqq4_w_pair(hqq4_q_pair(word, p), z2, s2);
+    *reinterpret_cast<uint4*>(w + n * K + 8 * j) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
 // ------------------------------------------------- base-3 ternary format --
 // (bonsai.h.)  A group's byte j holds the trits at group positions j, j+26,
 // j+52, j+78, j+104 as y = ceil(256 v / 243), v their base-3 number

@@ -125,13 +125,46 @@ int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const ui
                             int64_t N, int64_t K, int mode, uint16_t* out_host, uint16_t* A_dev,
                             uint16_t* out_dev, void* stream);
 
+/* ------------------------------------------ 4-bit group-affine weights --
+ * The pages name "4-bit HQQ" for the text encoder ("Cómo Bonsai Ternary 4B
+ * revoluciona la difusión texto-imagen", section "Arquitectura de despliegue
+ * y eficiencia en tiempo de ejecución") and nothing more.  This library
+ * reads it as HQQ's published scheme: an unsigned 4-bit q per weight and, per
+ * group of 64 weights along K, an FP16 scale s and an FP16 zero z, the weight
+ * being w = fp16(fp16(q - z) * s) (two IEEE FP16 operations).  The group
+ * size and the packing are this library's choices.
+ * Packed: rows of K/8 little-endian uint32 words; word j holds k = 8j..8j+7,
+ * weight i of it at bit 16 (i%2) + 4 (i/2) (weights 2p, 2p+1 at the same
+ * offset of the two 16-bit halves).  scales, zeros: FP16 [N, K/64].
+ * K must be a multiple of 128. */
+
+/* Bytes of packed 4-bit weights: N*K/2 (0 for an invalid shape). */
+size_t bonsai_hqq4_packed_bytes(int64_t N, int64_t K);
+
+/* q: uint8 [N,K] with values 0..15 -> packed.  Offline; synchronises
+ * `stream` to report BONSAI_ERR_BAD_CODE for a value above 15. */
+int bonsai_hqq4_pack(const uint8_t* q, int64_t N, int64_t K, void* packed, void* stream);
+
+/* Exact dequantisation: w = fp16(fp16(q - z) * s), FP16 [N,K] (bit-exact,
+ * IEEE rules for NaN, infinities and signed zeros). */
+int bonsai_hqq4_dequant(const void* packed, const uint16_t* scales, const uint16_t* zeros, int64_t N, int64_t K,
+                        uint16_t* w, void* stream);
+
+/* out[m,n] = fp16( sum_k A[m,k] * w[n,k] ) with the weights above, formed
+ * exactly as bonsai_hqq4_dequant forms them and summed in FP32 on the tensor
+ * cores; the same tiling, split and error behaviour as bonsai_lowbit_gemm.
+ * Weights that come out infinite or NaN give unspecified outputs. */
+int bonsai_hqq4_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, const uint16_t* zeros, int64_t M,
+                     int64_t N, int64_t K, uint16_t* out, void* stream);
+
 /* The launch bonsai_lowbit_gemm makes for this problem on the current
  * device: *block_t = tokens per tile (the MMA's N; each tile also covers 128
  * weight rows), *ksplit = CTAs that share one tile along K as a thread-block
  * cluster (1 = no split), *ctas = CTAs launched, *tiles = output tiles.
  * ctas < tiles x ksplit means the persistent form: one CTA per SM walks the
  * tiles tau = blockIdx, blockIdx + ctas, ...  Host-side only (queries
- * occupancy, launches nothing).  Zero-sized problems report zeros. */
+ * occupancy, launches nothing).  Zero-sized problems report zeros.  mode 4
+ * asks for the launch of bonsai_hqq4_gemm. */
 int bonsai_gemm_plan(int64_t M, int64_t N, int64_t K, int mode, int* block_t, int* ksplit, int* ctas,
                      int* tiles);
 

@@ -84,6 +84,13 @@ def test_argument_errors_before_any_device_work(lib):
     assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 128, 2, P, P) == 1
     assert lib.bonsai_lowbit_gemm(P, P, P, 4, 4, 128, 2, 8, P) == 3
     assert lib.bonsai_lowbit_gemm(P, P, P, 1 << 31, 4, 128, 2, 16, P) == 2
+    # 4-bit group-affine weights
+    assert lib.bonsai_hqq4_packed_bytes(8, 256) == 8 * 256 // 2 and lib.bonsai_hqq4_packed_bytes(8, 100) == 0
+    assert lib.bonsai_hqq4_pack(P, 4, 100, P, P) == 2
+    assert lib.bonsai_hqq4_pack(P, 4, 128, P, P) == 1
+    assert lib.bonsai_hqq4_dequant(16, 16, P, 4, 128, 16, P) == 1  # null zeros
+    assert lib.bonsai_hqq4_gemm(P, P, P, P, 0, 4, 128, P, P) == 0
+    assert lib.bonsai_hqq4_gemm(16, 16, 16, 24, 4, 4, 128, 16, P) == 3  # misaligned zeros
     # host-buffer form: A_host, packed, scales, M, N, K, mode, out_host, A_dev, out_dev, stream
     H = 16
     assert lib.bonsai_lowbit_gemm_host(H, H, H, 4, 4, 128, 0, H, H, H, P) == 1  # mode

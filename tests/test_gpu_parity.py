@@ -470,3 +470,75 @@ def test_bounded_wait_gives_up_and_reports():
                          dev(d["scales"].view(np.int16), torch.float16), "ternary")
     torch.cuda.synchronize()
     assert out.isfinite().all()
+
+
+# --------------------------------------- 4-bit group-affine weights (HQQ) --
+# Reading of the pages' "4-bit HQQ" (unpinned by the pages): w =
+# fp16(fp16(q - z) * s), groups of 64 along K.  Pack and dequant bit-exact,
+# the GEMM within the same tolerance as the other formats.
+def _hqq4_inputs(d):
+    q = dev(d["q"])
+    packed = bw.hqq4_pack(q)
+    return (packed, dev(d["scales"].view(np.int16), torch.float16), dev(d["zeros"].view(np.int16), torch.float16),
+            dev(d["A"].view(np.int16), torch.float16))
+
+
+@pytest.mark.parametrize("N,K", PACK_SHAPES)
+def test_hqq4_pack_and_dequant_bit_exact(oracle_mod, N, K):
+    d = workloads.make_hqq4(1, N, K, seed=N + K)
+    packed, s, z, _ = _hqq4_inputs(d)
+    ref_packed = oracle_mod.hqq4_pack(d["q"])
+    assert np.array_equal(to_u32(packed), ref_packed)
+    got = bw.hqq4_dequant(packed, s, z, K)
+    assert np.all(nan_aware_equal(to_u16(got), oracle_mod.hqq4_dequant(ref_packed, d["scales"], d["zeros"], K)))
+
+
+def test_hqq4_dequant_special_values(oracle_mod):
+    rng = np.random.default_rng(21)
+    N, K = 4096, 128
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    s = rng.integers(0, 65536, (N, 2)).astype(np.uint16)  # every kind of FP16: subnormal, inf, NaN, -0
+    z = rng.integers(0, 65536, (N, 2)).astype(np.uint16)
+    ref_packed = oracle_mod.hqq4_pack(q)
+    got = bw.hqq4_dequant(dev(ref_packed.view(np.int32)), dev(s.view(np.int16), torch.float16),
+                          dev(z.view(np.int16), torch.float16), K)
+    assert np.all(nan_aware_equal(to_u16(got), oracle_mod.hqq4_dequant(ref_packed, s, z, K)))
+
+
+def test_hqq4_pack_reports_bad_values():
+    q = np.full((64, 256), 3, np.uint8)
+    q[17, 200] = 16
+    with pytest.raises(bw.BonsaiError) as e:
+        bw.hqq4_pack(dev(q))
+    assert e.value.status == 4
+
+
+@pytest.mark.parametrize("M,N,K", SMALL_SHAPES + [(1357, 3880, 512), (700, 1000, 640), (16, 3072, 12288)])
+def test_hqq4_gemm_full(oracle_mod, M, N, K):
+    d = workloads.make_hqq4(M, N, K, seed=M + 5 * N + K)
+    packed, s, z, A = _hqq4_inputs(d)
+    out = bw.hqq4_gemm(A, packed, s, z)
+    torch.cuda.synchronize()
+    ref, _, absacc = oracle_mod.hqq4_gemm(d["A"], oracle_mod.hqq4_pack(d["q"]), d["scales"], d["zeros"], K)
+    assert_gemm_close(oracle_mod, to_u16(out), ref, absacc, f"hqq4 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(4608, 9216, 3072), (16, 3072, 9216)])
+def test_hqq4_gemm_full_size_sampled(oracle_mod, M, N, K):
+    d = workloads.make_hqq4(M, N, K, seed=77)
+    packed, s, z, A = _hqq4_inputs(d)
+    for _ in range(20):  # repeated launches: no device error, identical bits
+        out = bw.hqq4_gemm(A, packed, s, z)
+    first = bw.hqq4_gemm(A, packed, s, z)
+    torch.cuda.synchronize()
+    assert bw.get_device_error() == 0 and torch.equal(out, first)
+    rng = np.random.default_rng(M)
+    ms = np.unique(rng.integers(0, M, 48))
+    ns = np.unique(rng.integers(0, N, 256))
+    rows = oracle_mod.hqq4_dequant(oracle_mod.hqq4_pack(d["q"][ns]), d["scales"][ns], d["zeros"][ns], K)
+    ref, _, absacc = oracle_mod.gemm_w16(d["A"][ms], rows)
+    got = to_u16(first)[np.ix_(ms, ns)]
+    assert_gemm_close(oracle_mod, got, ref, absacc, f"hqq4 {M}x{N}x{K} sampled")
+    if M > 128:
+        plan = bw.gemm_plan(M, N, K, "hqq4")
+        assert plan["ctas"] < plan["tiles"], plan  # the persistent kernel

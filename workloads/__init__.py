@@ -118,6 +118,22 @@ def scales(rng: np.random.Generator, N: int, K: int) -> np.ndarray:
     return rng.uniform(0.005, 0.05, (N, K // GROUP)).astype(np.float16).view(np.uint16)
 
 
+def make_hqq4(M: int, N: int, K: int, seed: int):
+    """Inputs for the 4-bit group-affine weights: A (uint16 fp16 bits [M,K]),
+    q (uint8 [N,K], uniform on 0..15), scales ~ U[0.005, 0.05] and zeros ~
+    U[0, 15] (fp16 bits [N, K/64]), from the same spawned-stream scheme."""
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    ra, rc, rs = _streams(seed)
+    return {
+        "M": M, "N": N, "K": K,
+        "A": activations(ra, M, K),
+        "q": rc.integers(0, 16, (N, K), dtype=np.uint8),
+        "scales": rs.uniform(0.005, 0.05, (N, K // 64)).astype(np.float16).view(np.uint16),
+        "zeros": rs.uniform(0.0, 15.0, (N, K // 64)).astype(np.float16).view(np.uint16),
+    }
+
+
 def make(problem: Problem | None = None, *, mode=None, M=None, N=None, K=None, seed=None):
     """-> dict with A (uint16 fp16 bits [M,K]), codes (int8 [N,K]),
     scales (uint16 fp16 bits [N,K/128]) and the problem's sizes."""
