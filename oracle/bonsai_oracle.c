@@ -43,7 +43,9 @@
  * 64 weights along K an FP16 scale s and FP16 zero z, the weight being
  * evaluated in FP16 as w = fp16(fp16(q - z) * s).  The group size, the zero
  * as an FP16 value and the packing (oracle_hqq4_pack) are this reading's
- * choices; none of it is pinned by the pages.
+ * choices; none of it is pinned by the pages: parity unpinned for the
+ * oracle_hqq4_* functions (their FP16 arithmetic and layout are checked by
+ * the tests, the reading is not).
  */
 #include <math.h>
 #include <pthread.h>
