@@ -347,7 +347,7 @@ def test_narrow_tiles_repeated_launches(oracle_mod, mode, M, N, K):
 # full; the headline workload at sampled positions; back-to-back calls that
 # reuse the same work buffers.
 @pytest.mark.parametrize("mode,M,N,K", [("ternary", 1357, 3880, 512), ("binary", 16, 3072, 1024),
-                                        ("ternary", 300, 256, 384)])
+                                        ("ternary", 300, 256, 384), ("ternary_b3", 600, 384, 640)])
 def test_gemm_host_buffers_full(oracle_mod, mode, M, N, K):
     d = workloads.make(mode=mode, M=M, N=N, K=K, seed=7 * M + N + K)
     ref_packed = oracle_mod.pack(d["codes"], mode)
