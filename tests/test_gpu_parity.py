@@ -442,6 +442,29 @@ def test_gemm_empty_shapes():
     assert torch.equal(out, torch.zeros_like(out))
 
 
+@pytest.mark.parametrize("mode", MODES)
+def test_gemm_overflow_and_nan_match_the_oracle(oracle_mod, mode):
+    """Outputs beyond the FP16 range round to +-inf on both sides; a NaN
+    activation makes its whole output row NaN (every weight multiplies it)."""
+    M, N, K = 24, 256, 512
+    d = workloads.make(mode=mode, M=M, N=N, K=K, seed=31)
+    A = d["A"].copy()
+    A[:4] = np.float16(6.0e4).view(np.uint16)             # rows 0-3: huge activations -> overflow
+    A[4:8] = np.float16(-6.0e4).view(np.uint16)
+    A[8, 100] = np.uint16(0x7E00)                         # row 8: one NaN
+    scales = d["scales"].copy()
+    scales[:, :] = np.float16(0.5).view(np.uint16)
+    ref_packed, packed, _, _ = gpu_inputs(d, oracle_mod)
+    out = bw.lowbit_gemm(dev(A.view(np.int16), torch.float16), packed, dev(scales.view(np.int16), torch.float16),
+                         mode)
+    torch.cuda.synchronize()
+    ref, _, absacc = oracle_mod.gemm(A, ref_packed, scales, K, mode)
+    got = to_u16(out)
+    r = ref.view(np.float16)
+    assert np.isinf(r[:8]).any() and np.isnan(r[8]).all()  # the case is what it claims
+    assert_gemm_close(oracle_mod, got, ref, absacc, f"{mode} overflow / NaN")
+
+
 def test_gemm_zero_codes_and_zero_scales():
     K = 384
     A = torch.randn((40, K), dtype=torch.float16, device="cuda")
