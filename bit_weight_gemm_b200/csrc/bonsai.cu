@@ -1,6 +1,7 @@
 // bonsai.cu - the C ABI declared in include/bonsai.h: argument checks, tensor
-// maps, kernel selection and launches.  All arithmetic runs in the kernels of
-// pack_dequant.cuh and gemm_tc.cuh.
+// maps, kernel selection (the planner) and launches, and the host-buffer
+// pipeline.  All arithmetic runs in the kernels of pack_dequant.cuh,
+// gemm_tc.cuh and gemm_persistent.cuh.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

@@ -23,8 +23,9 @@
 //
 // The tensor core thus idles at a tile boundary only for the read-out of the
 // accumulator.  Requirements (checked by the host): more tiles than fit in one
-// wave, and K a multiple of 128 x the groups in one word stage (512 ternary,
-// 1024 binary), so that word stages never straddle two tiles.
+// wave, and K a multiple of 128 x max(4, groups in one word stage) (512 for
+// INT2, base-3 and 4-bit weights, 1024 binary), so that word stages never
+// straddle two tiles and every converter warp keeps its TMEM stage.
 #pragma once
 
 #include "gemm_tc.cuh"

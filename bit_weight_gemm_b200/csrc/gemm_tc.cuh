@@ -1,6 +1,8 @@
 // gemm_tc.cuh - fused dequantise + GEMM on the 5th-generation tensor cores.
 //
-// out[m,n] = sum_k A[m,k] * w[n,k],  w[n,k] = s[n,k/128] * t[n,k].
+// out[m,n] = sum_k A[m,k] * w[n,k],  w[n,k] = s[n,k/128] * t[n,k]  (binary,
+// ternary INT2, ternary base-3), or w = fp16(fp16(q - z) * s) with a scale
+// and zero per 64 weights (4-bit group-affine).
 //
 // A CTA computes a tile of 128 weight rows x BLOCK_T tokens over a range of
 // 128-wide K groups, as D^T = W * A^T, so that the weights are the MMA's M
@@ -9,17 +11,19 @@
 //   act ring   (warp 0)  TMA of the activation tile per group: BLOCK_T rows
 //                        x 128 FP16 as two 128-byte-swizzled K slices.
 //   word ring  (warp 2)  TMA of the 128 rows' packed words, 128 bytes of
-//                        each row per stage (4 ternary or 8 binary groups)
-//                        with 128-byte swizzling, so that the converters'
-//                        16-byte reads are free of bank conflicts and each
-//                        request moves a whole 128-byte line.
+//                        each row per stage (8 binary, 4 INT2 or 2 4-bit
+//                        groups) with 128-byte swizzling, so that the
+//                        converters' 16-byte reads are free of bank conflicts
+//                        and each request moves a whole 128-byte line; or one
+//                        unswizzled 112-byte base-3 block (4 groups).
 //   TMEM ring  (warps 3-18, four per TMEM lane quadrant, taking groups in
 //                        turn) converters: each thread owns one weight row,
-//                        turns the group's words into exact FP16 products
-//                        (binary: sign bit over s; ternary INT2: the shifted
-//                        2-bit field is 2t, times s; base-3: digits stepped
-//                        out of two bytes at a time, t, times s) and writes
-//                        them to a TMEM stage with tcgen05.st.
+//                        turns the group's words into FP16 weights (binary:
+//                        sign bit over s; ternary INT2: the shifted 2-bit
+//                        field is 2t, times s; base-3: digits stepped out of
+//                        two bytes at a time, t, times s; 4-bit: the nibble
+//                        pair under FP16's 1024, minus 1024, minus z, times
+//                        s) and writes them to a TMEM stage with tcgen05.st.
 //   warp 1               allocates TMEM; one thread issues
 //                        tcgen05.mma.kind::f16 (M=128, N=BLOCK_T, K=16) x 8
 //                        per group, A from TMEM, B from shared memory, FP32
@@ -31,7 +35,8 @@
 // for that kernel's completion before its first global-memory access.
 //
 // Epilogue, one CTA per tile (ksplit = 1): the converters read the
-// accumulator (tcgen05.ld), scale by 1 (binary) or 1/2 (ternary, exact),
+// accumulator (tcgen05.ld), scale by 1/2 (INT2, which converts 2ts; exact)
+// or 1,
 // round once to FP16 into a shared-memory tile, and one TMA store writes it.
 // Split K (ksplit > 1, small M): the ksplit CTAs of a cluster share a tile;
 // each leaves its FP32 partial in shared memory and, after a cluster
@@ -40,8 +45,9 @@
 // and stores it.  Accumulation is spread over several TMEM accumulators so
 // that narrow MMAs do not queue behind one accumulator.
 //
-// Weights are multiplied exactly: |t| <= 1 and s is FP16, so s*t (and 2*s*t
-// for |s| < 32768) is an FP16 value; the sum runs in FP32.
+// Weights are formed exactly: |t| <= 1 and s is FP16, so s*t (and 2*s*t for
+// |s| < 32768) is an FP16 value, and the 4-bit weight is by definition the
+// FP16 result of its two FP16 operations; products and the sum run in FP32.
 #pragma once
 
 #include "pack_dequant.cuh"

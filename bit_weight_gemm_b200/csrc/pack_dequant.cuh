@@ -1,4 +1,7 @@
-// pack_dequant.cuh - bit packing of weight codes and exact dequantisation.
+// pack_dequant.cuh - bit packing of weight codes and exact dequantisation, for
+// the binary and INT2 formats (below), the 4-bit group-affine weights and the
+// base-3 ternary format (their sections further down), with the decode
+// helpers the GEMM converters share.
 //
 // Both kernels are elementwise and bound by HBM bandwidth: one thread owns a
 // few consecutive packed words, reads their codes (or writes their weights)
