@@ -99,9 +99,8 @@ struct GemmTile {
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   // (4-bit group-affine weights keep scale and zero pairs in registers.)
   static constexpr int kScaleBytes = (BLOCK_T >= 256 || kHqq) ? 0 : 32768;
-  // Converter warps: 2 or 4 per TMEM lane quadrant.  (Five per quadrant on
-  // narrow tiles measured 2-5% slower: their tensor-memory stores, not the
-  // number of groups in conversion, set the pace.)
+  // Converter warps: four per TMEM lane quadrant.  (Five per quadrant on
+  // narrow tiles measured 2-5% slower.)
   static constexpr int kConvWarps = 16;
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
   // Epilogue: the quadrant's warps split the token columns, 8 at least each:
