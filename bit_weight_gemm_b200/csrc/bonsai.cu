@@ -211,16 +211,19 @@ int smem_opt_in(int bytes) {
   return BONSAI_OK;
 }
 
-// Clusters of `ksplit` CTAs that can be resident at once (0 if unknown).
+// Clusters of `ksplit` CTAs that can be resident at once on the current
+// device (0 if unknown).
 template <int MODE, int BLOCK_T>
 int resident_clusters(int ksplit) {
   using T = GemmTile<MODE, BLOCK_T>;
   static std::mutex mu;
-  static int cache[9] = {0};
+  static int cache[64][9] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   std::lock_guard<std::mutex> lock(mu);
   if (ksplit < 1 || ksplit > 8) return 0;
   if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T>>(T::kSmemBytes) != BONSAI_OK) return 0;
-  if (cache[ksplit] == 0) {
+  if (cache[dev][ksplit] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, ksplit);
     cfg.blockDim = dim3(T::kThreads);
@@ -237,9 +240,9 @@ int resident_clusters(int ksplit) {
       cudaGetLastError();
       n = -1;
     }
-    cache[ksplit] = n;
+    cache[dev][ksplit] = n;
   }
-  return cache[ksplit] > 0 ? cache[ksplit] : 0;
+  return cache[dev][ksplit] > 0 ? cache[dev][ksplit] : 0;
 }
 
 template <int MODE, int BLOCK_T>

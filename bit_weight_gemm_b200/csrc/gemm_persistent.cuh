@@ -115,7 +115,6 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
   auto tile_n0 = [&](int it) { return ((blockIdx.x + it * gridDim.x) % args.tiles_n) * T::kRows; };
   auto tile_m0 = [&](int it) { return static_cast<int>((blockIdx.x + it * gridDim.x) / args.tiles_n) * T::kBlockT; };
 
-  if (threadIdx.x == 0) griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < AS; ++s) {
       mbar_init(act_full0 + 8 * s, 1);
@@ -146,6 +145,10 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
+  // Dependents may launch once this CTA holds its tensor memory (see
+  // lowbit_gemm_kernel: a dependent CTA may wait for these columns, never the
+  // reverse).
+  if (threadIdx.x == 0) griddep_launch_dependents();
   griddep_wait();
 
   if (warp == 0) {

@@ -316,9 +316,6 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
   const int ng = g_end - g_begin;
   const uint64_t limit = args.wait_limit_ns;
 
-  // The next launch in the stream may start its own prologue now; it waits
-  // (griddep_wait) for this grid to finish before touching global memory.
-  if (threadIdx.x == 0) griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < AS; ++s) {
       mbar_init(act_full0 + 8 * s, 1);
@@ -359,6 +356,13 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);  // warp-uniform (see above)
+  // The next launch in the stream may start its own prologue now; it waits
+  // (griddep_wait) for this grid to finish before touching global memory.
+  // Only now, with this CTA's tensor memory held: a dependent CTA placed on
+  // this SM may then block in its own allocation until this CTA frees its
+  // columns, but never the other way round (this CTA waits on nothing the
+  // dependent holds), so the two cannot deadlock.
+  if (threadIdx.x == 0) griddep_launch_dependents();
   // Everything above touched only this CTA's own resources; global memory
   // (activations, weights, scales, output) only after the preceding grid in
   // the stream has completed.
@@ -412,6 +416,11 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       for (int i = issued > WS ? issued - WS : 0; i < issued; ++i) {
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(w_full0 + 8 * (i % WS), (i / WS) & 1) && global_timer_ns() - t0 < limit) {
+        }
+      }
+      if (args.scale_box > 0) {  // the scale tile's copy, which the converters may not have waited for
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(s_full, 0) && global_timer_ns() - t0 < limit) {
         }
       }
     }

@@ -1,9 +1,14 @@
 // ptx.cuh - thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads,
 // tensor-memory allocation, tcgen05 MMA / load / store, and bounded waits.
 //
-// Every wait in the library goes through wait_phase(), which gives up after a
-// time limit, records BONSAI_ERR_TIMEOUT in the device error word and raises
-// the CTA's abort flag so the other warps stop too.  No wait can spin forever.
+// Every mbarrier wait in the library goes through wait_phase(), which gives
+// up after a time limit, records BONSAI_ERR_TIMEOUT in the device error word
+// and raises the CTA's abort flag so the other warps stop too.  The one
+// blocking instruction without a limit is tcgen05.alloc, which waits for free
+// tensor-memory columns.  It cannot wait forever: every kernel allocates
+// before it lets dependent grids launch (griddepcontrol.launch_dependents)
+// and frees its columns before it exits, and a CTA holding columns waits only
+// for grids launched before it, whose CTAs already hold theirs.
 #pragma once
 
 #include <cuda.h>

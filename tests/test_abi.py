@@ -51,10 +51,14 @@ def test_library_does_not_need_libcuda(lib):
     assert "libcuda.so" not in out  # driver calls go through the runtime's entry-point lookup
 
 
-def test_library_is_built_for_sm100a(lib):
-    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", bw.library_path()], capture_output=True,
-                         text=True).stdout
-    assert "sm_100a" in out
+def test_library_is_built_for_sm100a():
+    """The build compiles for sm_100a and nothing else (the kernels use
+    tcgen05 and TMA; a device of another architecture is refused at run
+    time with BONSAI_ERR_ARCH)."""
+    cmd = bw_build.command()
+    gencodes = [cmd[i + 1] for i, a in enumerate(cmd) if a == "-gencode"]
+    assert gencodes == ["arch=compute_100a,code=sm_100a"]
+    assert not any(a.startswith(("-arch", "--gpu-architecture")) for a in cmd)
 
 
 def test_sizes(lib):
