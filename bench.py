@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 WORKLOAD = workloads.TERNARY_MLP_UP_4608
-SMALL = workloads.TERNARY_MLP_DOWN_16
+SMALL = [workloads.TERNARY_MLP_DOWN_16, workloads.TERNARY_QKV_16]
 METRIC = "low-bit W.A GEMM TFLOP/s (M=4608,K=3072,N=9216 ternary)"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -367,7 +367,7 @@ def run_bonsai(args):
 
     small = None
     if not args.no_extras or args.small_only:
-        small = time_small(torch, bw, SMALL, args, dist, peaks, peaks_kind)
+        small = [time_small(torch, bw, sp, args, dist, peaks, peaks_kind) for sp in SMALL]
     stack = None
     if not args.no_extras and not args.small_only:
         stack = [time_stack(torch, bw, m, "ternary", 20, 3) for m in (4608, 1024)]
@@ -476,7 +476,7 @@ def time_formats(torch, bw, args, dist, peaks, peaks_kind):
     in the base-3 format (1.75 bits per weight against INT2's 2): TFLOP/s at
     M=4608 and GB/s of algorithmic bytes (fewer packed bytes) at M=16."""
     out = []
-    for base, sets_n, unit in ((WORKLOAD, args.sets, "TFLOP/s"), (SMALL, 64, "GB/s")):
+    for base, sets_n, unit in ((WORKLOAD, args.sets, "TFLOP/s"), (SMALL[0], 64, "GB/s")):
         p = workloads.Problem("base-3 " + base.name, "ternary_b3", base.M, base.N, base.K, base.seed)
         sets = make_sets(p, sets_n, torch, bw, distinct_weights=False)
         steps = max(200, min(args.steps, 2000))

@@ -11,6 +11,7 @@
 
 #include "bonsai.h"
 #include "gemm_persistent.cuh"
+#include "gemm_small.cuh"
 #include "gemm_tc.cuh"
 #include "pack_dequant.cuh"
 
@@ -368,6 +369,111 @@ int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t
   return launch_status();
 }
 
+// Clusters of `ksplit` small-M CTAs that can be resident at once on the
+// current device (the kernel takes one SM per CTA; clusters must fit within
+// a GPC, so fewer than SMs / ksplit may fit).  0 if unknown.
+template <int MODE>
+int small_resident_clusters(int ksplit) {
+  using T = SmallTile<MODE>;
+  static std::mutex mu;
+  static int cache[64][9] = {};
+  int dev = 0;
+  if (ksplit < 1 || ksplit > T::kMaxSplit) return 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (smem_opt_in<lowbit_gemm_small_kernel<MODE>>(T::kSmemBytes) != BONSAI_OK) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev][ksplit] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, ksplit);
+    cfg.blockDim = dim3(T::kThreads);
+    cfg.dynamicSmemBytes = T::kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 1;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = ksplit;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, lowbit_gemm_small_kernel<MODE>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = -1;
+    }
+    cache[dev][ksplit] = n;
+  }
+  return cache[dev][ksplit] > 0 ? cache[dev][ksplit] : 0;
+}
+
+// Small-M form (gemm_small.cuh): the K split for up to 16 tokens, 0 when the
+// form does not apply.  Every CTA's range must fit its shared memory
+// (kMaxGroups groups); among the splits that allow it, the largest whose
+// tiles x ksplit CTAs are all resident at once (one wave), else the
+// smallest.
+template <int MODE>
+int small_ksplit(int M, int N, int K) {
+  using T = SmallTile<MODE>;
+  if constexpr (MODE == kModeHqq4) return 0;  // (its weights are formed with the scale, in the other kernels)
+  if (M > T::kBlockT) return 0;
+  const int groups = K / kGroup;
+  const int tiles = (N + T::kRows - 1) / T::kRows;
+  int best = 0;
+  bool best_fits = false;
+  for (int ks = 1; ks <= T::kMaxSplit && ks * T::kGroupAlign <= (groups > T::kGroupAlign ? groups : T::kGroupAlign);
+       ++ks) {
+    int widest = 0;
+    for (int z = 0; z < ks; ++z) {
+      const int w = split_bound<T::kGroupAlign>(z + 1, groups, ks) - split_bound<T::kGroupAlign>(z, groups, ks);
+      if (w < 1) widest = 1 << 30;  // an empty range
+      widest = w > widest ? w : widest;
+    }
+    if (widest > T::kMaxGroups) continue;
+    const int resident = ks == 1 ? sm_count() : small_resident_clusters<MODE>(ks);
+    if (tiles <= resident) {  // one wave: the largest such split wins
+      best = ks;
+      best_fits = true;
+    } else if (!best_fits && best == 0) {  // none in one wave (yet): the smallest feasible split
+      best = ks;
+    }
+  }
+  return best;
+}
+
+template <int MODE>
+int launch_gemm_small(const uint16_t* A, const void* packed, const uint16_t* scales, int M, int N, int K, int ksplit,
+                      uint16_t* out, cudaStream_t stream) {
+  using T = SmallTile<MODE>;
+  auto kernel = lowbit_gemm_small_kernel<MODE>;
+  if (smem_opt_in<lowbit_gemm_small_kernel<MODE>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
+  CUtensorMap map_act, map_w;
+  if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, T::kBlockT, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BONSAI_ERR_CUDA;
+  if (!make_weight_map(&map_w, packed, N, K, MODE)) return BONSAI_ERR_CUDA;
+  SmallArgs args;
+  args.scales = scales;
+  args.out = out;
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.ksplit = ksplit;
+  args.wait_limit_ns = kDefaultWaitLimitNs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((N + T::kRows - 1) / T::kRows, 1, ksplit);
+  cfg.blockDim = dim3(T::kThreads);
+  cfg.dynamicSmemBytes = T::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  attrs[1].id = cudaLaunchAttributeClusterDimension;
+  attrs[1].val.clusterDim.x = 1;
+  attrs[1].val.clusterDim.y = 1;
+  attrs[1].val.clusterDim.z = ksplit;
+  cfg.attrs = attrs;
+  cfg.numAttrs = ksplit > 1 ? 2 : 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, map_act, map_w, args) != cudaSuccess) return BONSAI_ERR_CUDA;
+  return launch_status();
+}
+
 // ------------------------------------------------------------- planning --
 // Launch costs in microseconds, measured on a B200 with an M sweep of single
 // launches (16..4608 tokens on the MMDiT layer shapes, clocks under the power
@@ -391,6 +497,7 @@ constexpr double kPersistentBoundary = 1.0;
 struct Plan {
   int block_t = 0, ksplit = 0, ctas = 0, tiles = 0;
   bool persistent = false;
+  bool small = false;  // the bandwidth-bound form of gemm_small.cuh
   double cost = 1e30;
 };
 
@@ -430,6 +537,14 @@ void consider(int M, int N, int K, Plan* best) {
 template <int MODE>
 Plan plan_gemm(int M, int N, int K) {
   Plan best;
+  if (const int ks = small_ksplit<MODE>(M, N, K)) {
+    best.block_t = SmallTile<MODE>::kBlockT;
+    best.ksplit = ks;
+    best.tiles = (N + 127) / 128;
+    best.ctas = best.tiles * ks;
+    best.small = true;
+    return best;
+  }
   if (M <= 16) {
     consider<MODE, 16>(M, N, K, &best);
   } else if (M <= 32) {
@@ -450,6 +565,8 @@ int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales,
                   int K,
                   uint16_t* out, cudaStream_t stream) {
   const Plan p = plan_gemm<MODE>(M, N, K);
+  if constexpr (MODE != kModeHqq4)
+    if (p.small) return launch_gemm_small<MODE>(A, packed, scales, M, N, K, p.ksplit, out, stream);
   if (p.persistent) return launch_gemm_persistent<MODE>(A, packed, scales, zeros, M, N, K, out, stream);
   switch (p.block_t) {
     case 16: return launch_gemm<MODE, 16>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);

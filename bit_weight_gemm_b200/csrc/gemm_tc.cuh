@@ -237,7 +237,7 @@ __device__ __forceinline__ void convert_group_hqq4(const uint32_t* words, uint32
 // Boundary z of a split of `groups` into `ks` ranges, on multiples of ALIGN
 // (nearest); the caller keeps ks <= groups / ALIGN so that no range is empty.
 template <int ALIGN>
-__device__ __forceinline__ int split_bound(int z, int groups, int ks) {
+__host__ __device__ __forceinline__ int split_bound(int z, int groups, int ks) {
   if (z >= ks) return groups;
   const int x = static_cast<int>(static_cast<int64_t>(z) * groups / ks);
   const int r = (x + ALIGN / 2) / ALIGN * ALIGN;

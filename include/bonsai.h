@@ -78,22 +78,42 @@ size_t bonsai_packed_bytes(int64_t N, int64_t K, int mode);
 /* Bytes of the FP16 scales for an [N,K] weight: 2*N*K/128. */
 size_t bonsai_scale_bytes(int64_t N, int64_t K);
 
-/* Pack weight codes.  codes: int8 [N,K] with every value in the mode's
- * alphabet; packed: bonsai_packed_bytes(N,K,mode) bytes, written in the
- * format above.  This call is offline (once per weight): it synchronises
- * `stream` before returning so that it can report BONSAI_ERR_BAD_CODE when a
- * code is outside the alphabet (packed is then unspecified).  Concurrent
+/* Pack weight codes.  The alphabets and bit counts come from the pages:
+ * ternary t in {-1,0,+1} stored as INT2, two bits per weight, for CUDA ("Cómo
+ * Bonsai Ternary 4B revoluciona la difusión texto-imagen", section
+ * "Representación y almacenamiento de los pesos ternarios"); binary t in
+ * {-1,+1} at one bit, 1.125 effective bits per weight with the group scale
+ * ("Bonsai Image 4B 1-bit untuk pembuatan gambar di perangkat lokal",
+ * section "Bonsai Image 4B untuk pembuatan gambar lokal").  The bit layout
+ * is this library's.
+ * codes: int8 [N,K] with every value in the mode's alphabet; packed:
+ * bonsai_packed_bytes(N,K,mode) bytes, written in the format above.  This
+ * call is offline (once per weight): it synchronises `stream` before
+ * returning so that it can report BONSAI_ERR_BAD_CODE when a code is outside
+ * the alphabet (packed is then unspecified).  Concurrent
  * bonsai_pack calls on different streams share the flag that reports it. */
 int bonsai_pack(const int8_t* codes, int64_t N, int64_t K, int mode, void* packed, void* stream);
 
 /* Exact dequantisation: w[n,k] = fp16(t[n,k] * s[n,k/128]), the IEEE
- * product (bit-exact: +-s, +-0, or NaN for 0*inf and NaN scales).
+ * product (bit-exact: +-s, +-0, or NaN for 0*inf and NaN scales).  This is
+ * the pages' weight equation w_i = scale_g * t_i with one FP16 scale per
+ * group of 128 weights ("Cómo Bonsai Ternary 4B revoluciona la difusión
+ * texto-imagen", section "Representación y almacenamiento de los pesos
+ * ternarios").
  * packed: as written by bonsai_pack; scales: FP16 [N,K/128]; w: FP16 [N,K].
  * Meant for testing and for callers that want a dense copy. */
 int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_t K, int mode,
                    uint16_t* w, void* stream);
 
 /* The fused low-bit GEMM: out[m,n] = fp16( sum_k A[m,k] * w[n,k] ).
+ * This is the quantised linear layer of the pages: every matmul-heavy linear
+ * of the diffusion transformer (Q/K/V projections, MLP weights, the
+ * double-stream add-K/Q/V linears) holds such weights ("Cómo Bonsai Ternary
+ * 4B revoluciona la difusión texto-imagen", section "Representación y
+ * almacenamiento de los pesos ternarios"), and the transformer runs once per
+ * denoising step, so its weight bandwidth sets the step's speed
+ * ("Introducing 1-bit and Ternary Bonsai Image 4B: Image Generation for
+ * Local Devices", section "端侧约束：为什么 diffusion transformer 是唯一值得压缩的部分").
  * A: FP16 [M,K]; packed/scales: as above for an [N,K] weight; out: FP16
  * [M,N].  Products are formed exactly and summed in FP32 on the tensor
  * cores, then rounded once to FP16 (nearest even).  Scales must be finite
@@ -119,6 +139,10 @@ int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* sc
  * and everything enqueued on `stream` afterwards is ordered after it; the
  * call returns without synchronising.  Host buffers must stay valid and
  * unmodified (A_host) / unread (out_host) until `stream` reaches that point.
+ * Concurrency: every call on one device uses the same three library streams
+ * (and one process-wide lock while it enqueues), so calls made from several
+ * threads or user streams run one after another on the GPU, never
+ * overlapped with each other.
  * Errors: as bonsai_lowbit_gemm, plus BONSAI_ERR_INVALID_ARG for null
  * pointers. */
 int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const uint16_t* scales, int64_t M,
