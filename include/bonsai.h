@@ -121,7 +121,13 @@ int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_
  * FP16); outside that range the result is unspecified.  out must not
  * overlap A, packed or scales.  An INT2 field with the pattern 10 (not a
  * ternary code) contributes zero; a base-3 byte that is not a code gives
- * unspecified values for its five weights. */
+ * unspecified values for its five weights.
+ * Stream order: A is read, and out written, only after everything enqueued
+ * before the call on `stream` has completed.  packed and scales, however, are
+ * read-only weights and may be read as soon as the launch starts, which for
+ * M <= 16 overlaps the end of the kernel enqueued just before it: that
+ * kernel must not write packed or scales (work enqueued earlier may; so may
+ * bonsai_pack, which returns only after its writes are complete). */
 int bonsai_lowbit_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, int64_t M,
                        int64_t N, int64_t K, int mode, uint16_t* out, void* stream);
 
