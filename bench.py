@@ -53,6 +53,13 @@ def parse_args():
     ap.add_argument("--sets", type=int, default=4, help="rotating input sets (their sum exceeds L2)")
     ap.add_argument("--no-extras", action="store_true", help="skip small-M, e2e, CPU baseline, clocks")
     ap.add_argument("--small-only", action="store_true", help="time only the M=16 workload (for profiling)")
+    ap.add_argument("--offline-only", action="store_true", help="time only pack and dequant (for profiling)")
+    ap.add_argument("--layers-only", action="store_true", help="time only the single-stream layer shapes")
+    ap.add_argument("--case", default=None,
+                    help="run one configuration --launches times, untimed (the command the committed ncu summaries "
+                         "profile): MODE:M:N:K for the GEMM (MODE binary, ternary, ternary_b3 or hqq4), "
+                         "pack-MODE:N:K or dequant-MODE:N:K")
+    ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--m-sweep", action="store_true",
                     help="time the GEMM over M = 16..4608 on the stack's five layer shapes and print one JSON line")
     return ap.parse_args()
@@ -374,11 +381,16 @@ def run_bonsai(args):
         stack.append(time_stack(torch, bw, 4608, "ternary", 20, 3, split_qkv=True))
         stack += [time_stack(torch, bw, None, "ternary", 20, 3, streams=st) for st in ((4096, 512), (1024, 512))]
         stack += [time_stack(torch, bw, m, "binary", 20, 3) for m in (4608, 1024)]
+    layers = None
+    if not args.no_extras and not args.small_only:
+        layers = time_layers(torch, bw, args, dist)
     cublas = None
     formats = None
+    offline = None
     if not args.no_extras and not args.small_only:
         cublas = cublas_fp16_same_run(torch)
         formats = time_formats(torch, bw, args, dist, peaks, peaks_kind)
+        offline = time_pack_dequant(torch, bw, p, peaks, peaks_kind)
 
     if dist is not None:
         dist.barrier()
@@ -406,7 +418,9 @@ def run_bonsai(args):
                 "cpu_baseline": cpu,
                 "small_m": small,
                 "stack": stack,
+                "layers": layers,
                 "formats": formats,
+                "pack_dequant": offline,
             }
             print(json.dumps(line), flush=True)
     if dist is not None:
@@ -524,6 +538,105 @@ def time_formats(torch, bw, args, dist, peaks, peaks_kind):
     out.append({"workload": "4-bit group-affine " + p.name, "mode": "hqq4", "M": p.M, "N": p.N, "K": p.K,
                 "value": flops(p) / t / 1e12, "unit": "TFLOP/s", "us_per_launch": t * 1e6,
                 "packed_bytes": p.N * p.K // 2, "plan": bw.gemm_plan(p.M, p.N, p.K, "hqq4")})
+    return out
+
+
+LAYER_SHAPES = ((18432, 3072, "single-stream fused QKV + MLP-up"), (3072, 12288, "single-stream out"))
+
+
+def time_layers(torch, bw, args, dist):
+    """The single-stream layers of the stack on their own, at the token counts
+    of a 1024^2 image + text (4608), a 512^2 image + text (1536) and a 512^2
+    image (1024): TFLOP/s of single launches (rotating inputs above L2,
+    CUDA-graph replay) with the launch the planner chose."""
+    out = []
+    for n, k, name in LAYER_SHAPES:
+        for m in (4608, 1536, 1024):
+            p = workloads.Problem(f"{name} M={m}", "ternary", m, n, k, 5000 + m + n)
+            count = int(min(16, max(2, -(-4 * 126 * 2 ** 20 // algorithmic_bytes(p)))))
+            sets = make_sets(p, count, torch, bw, distinct_weights=False)
+            steps = max(count * 8, 200) // count * count
+            secs = time_launches(torch, bw, p, sets, steps, 3, dist)
+            t = max_over_ranks(torch, secs, dist) / steps
+            del sets
+            out.append({"layer": name, "M": m, "N": n, "K": k, "us_per_launch": t * 1e6, "tflops": flops(p) / t / 1e12,
+                        "plan": bw.gemm_plan(m, n, k, "ternary")})
+    return out
+
+
+def time_pack_dequant(torch, bw, p, peaks, peaks_kind, sets=5, reps=20):
+    """The offline pack and the test-facing dequant on the headline weight
+    shape, in GB/s of their algorithmic bytes (codes in + packed words out;
+    packed words + scales in + FP16 weights out) against the measured HBM
+    copy bandwidth.  bonsai_pack synchronises to read its bad-code flag, so
+    its figure is per call (CUDA events around the call: flag reset, kernel,
+    flag read-back), the median of `reps` calls over `sets` rotating inputs
+    (larger than L2); dequant is timed as back-to-back launches replayed from
+    a CUDA graph."""
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out = []
+    def call_time(codes, packed, mode):
+        """Median per-call time of bonsai_pack over rotating inputs."""
+        times = []
+        for i in range(reps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            bw.pack(codes[i % len(codes)], mode, out=packed[i % len(codes)])
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                times.append(e0.elapsed_time(e1) / 1e3)
+        return statistics.median(times)
+
+    for mode in ("ternary", "binary", "ternary_b3"):
+        d = workloads.make(mode=mode, M=1, N=p.N, K=p.K, seed=p.seed)
+        codes = [torch.from_numpy(d["codes"]).cuda() for _ in range(sets)]
+        packed = [bw.pack(c, mode) for c in codes]
+        t1 = call_time(codes, packed, mode)
+        # Kernel time: one call on a weight 16 times as tall (453 MB of codes
+        # for the headline shape, so the kernel dominates) minus the fixed
+        # cost of a call (flag reset, read-back, synchronisation) measured on
+        # a one-group weight, divided by 16.
+        tiny = [torch.from_numpy(d["codes"][:8, :128].copy()).cuda() for _ in range(2)]
+        t0 = call_time(tiny, [bw.pack(c, mode) for c in tiny], mode)
+        big = [c.repeat(16, 1) for c in codes[:2]]
+        big_packed = [bw.pack(c, mode) for c in big]
+        t16 = call_time(big, big_packed, mode)
+        del big, big_packed
+        t = (t16 - t0) / 16
+        nbytes = p.N * p.K + packed_weight_bytes(mode, p.N, p.K)
+        out.append({"op": "pack", "mode": mode, "N": p.N, "K": p.K, "us_kernel": t * 1e6, "us_per_call": t1 * 1e6,
+                    "value": nbytes / t / 1e9, "unit": "GB/s", "frac": nbytes / t / 1e9 / peak,
+                    "algorithmic_bytes": nbytes,
+                    "timing": "kernel time = (call on a 16x taller weight - call on one group) / 16; per call "
+                              "incl. flag reset/read-back and synchronisation; CUDA events, medians"})
+        if mode == "ternary_b3":
+            continue
+        scales = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+        sets_dq = [(packed[j], scales.clone(), torch.empty((p.N, p.K), dtype=torch.float16, device="cuda"))
+                   for j in range(3)]
+        for pk, sc, w in sets_dq:
+            bw.dequant(pk, sc, p.K, mode, out=w)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for pk, sc, w in sets_dq:
+                bw.dequant(pk, sc, p.K, mode, out=w)
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / (reps * len(sets_dq))
+        del graph, sets_dq
+        nbytes = packed_weight_bytes(mode, p.N, p.K) + 2 * p.N * (p.K // 128) + 2 * p.N * p.K
+        out.append({"op": "dequant", "mode": mode, "N": p.N, "K": p.K, "us_per_launch": t * 1e6,
+                    "value": nbytes / t / 1e9, "unit": "GB/s", "frac": nbytes / t / 1e9 / peak,
+                    "algorithmic_bytes": nbytes, "timing": "CUDA graph replay, CUDA events"})
+        del codes, packed
     return out
 
 
@@ -658,10 +771,81 @@ def run_m_sweep(args):
     return 0
 
 
+def run_offline(args):
+    """Pack and dequant alone (for profiling): one JSON line."""
+    import torch
+
+    torch.cuda.set_device(0)
+    import bit_weight_gemm_b200 as bw
+
+    peaks, peaks_kind = load_peaks()
+    res = time_pack_dequant(torch, bw, WORKLOAD, peaks, peaks_kind)
+    assert bw.get_device_error() == 0
+    print(json.dumps({"pack_dequant": res, "peak_source": f"{peaks_kind} hbm copy"}), flush=True)
+    return 0
+
+
+def run_case(args):
+    """One configuration of one kernel, launched --launches times on the
+    seeded workload inputs: the command line the ncu summaries under
+    profiles/ profile."""
+    import torch
+
+    torch.cuda.set_device(0)
+    import bit_weight_gemm_b200 as bw
+
+    op, _, rest = args.case.rpartition("-") if args.case.split(":")[0].startswith(("pack-", "dequant-")) else \
+        ("gemm", "", args.case)
+    fields = rest.split(":")
+    mode = fields[0]
+    if op == "gemm":
+        M, N, K = (int(x) for x in fields[1:4])
+    else:
+        M, (N, K) = 1, (int(x) for x in fields[1:3])
+    if mode == "hqq4":
+        d = workloads.make_hqq4(M, N, K, seed=7)
+        packed = bw.hqq4_pack(torch.from_numpy(d["q"]).cuda())
+        s = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+        z = torch.from_numpy(d["zeros"].view(np.int16)).view(torch.float16).cuda()
+        A = torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).cuda()
+        run = {"gemm": lambda: bw.hqq4_gemm(A, packed, s, z),
+               "dequant": lambda: bw.hqq4_dequant(packed, s, z, K),
+               "pack": lambda: bw.hqq4_pack(torch.from_numpy(d["q"]).cuda())}[op]
+    else:
+        d = workloads.make(mode=mode, M=M, N=N, K=K, seed=7)
+        codes = torch.from_numpy(d["codes"]).cuda()
+        packed = bw.pack(codes, mode)
+        s = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
+        A = torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).cuda()
+        run = {"gemm": lambda: bw.lowbit_gemm(A, packed, s, mode),
+               "dequant": lambda: bw.dequant(packed, s, K, mode),
+               "pack": lambda: bw.pack(codes, mode, out=packed)}[op]
+    torch.cuda.synchronize()
+    for _ in range(args.launches):
+        run()
+    torch.cuda.synchronize()
+    assert bw.get_device_error() == 0
+    plan = bw.gemm_plan(M, N, K, mode) if op == "gemm" else None
+    print(json.dumps({"case": args.case, "launches": args.launches, "plan": plan}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.case:
+        return run_case(args)
     if args.m_sweep:
         return run_m_sweep(args)
+    if args.offline_only:
+        return run_offline(args)
+    if args.layers_only:
+        import torch
+
+        torch.cuda.set_device(0)
+        import bit_weight_gemm_b200 as bw
+
+        print(json.dumps({"layers": time_layers(torch, bw, args, None)}), flush=True)
+        return 0
     if args.impl == "reference":
         return run_reference(args)
     return run_bonsai(args)

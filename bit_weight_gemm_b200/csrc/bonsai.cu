@@ -321,11 +321,11 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, c
   return launch_status();
 }
 
-// Persistent form (gemm_persistent.cuh): more 256-token tiles than SMs and
-// whole word stages per tile.
-template <int MODE>
+// Persistent form (gemm_persistent.cuh): more BLOCK_T-token tiles than SMs
+// and whole word stages per tile.
+template <int MODE, int BLOCK_T>
 bool use_persistent(int M, int N, int K) {
-  using T = PersistTile<MODE>;
+  using T = PersistTile<MODE, BLOCK_T>;
   // Whole word stages per tile, and a group count per tile that is a
   // multiple of 4 (each converter warp keeps its TMEM stage across tiles).
   const int per_stage = T::kWGroups > 4 ? T::kWGroups : 4;
@@ -334,13 +334,13 @@ bool use_persistent(int M, int N, int K) {
   return tiles > sm_count();
 }
 
-template <int MODE>
+template <int MODE, int BLOCK_T>
 int launch_gemm_persistent(const uint16_t* A, const void* packed, const uint16_t* scales, const uint16_t* zeros, int M,
                            int N, int K,
                            uint16_t* out, cudaStream_t stream) {
-  using T = PersistTile<MODE>;
-  auto kernel = lowbit_gemm_persistent_kernel<MODE>;
-  if (smem_opt_in<lowbit_gemm_persistent_kernel<MODE>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
+  using T = PersistTile<MODE, BLOCK_T>;
+  auto kernel = lowbit_gemm_persistent_kernel<MODE, BLOCK_T>;
+  if (smem_opt_in<lowbit_gemm_persistent_kernel<MODE, BLOCK_T>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
   CUtensorMap map_act, map_w;
   if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, T::kBlockT, CU_TENSOR_MAP_SWIZZLE_128B))
     return BONSAI_ERR_CUDA;
@@ -489,6 +489,7 @@ constexpr TileCost tile_cost(int block_t) {
   return block_t <= 32    ? TileCost{0.31, 1.5, 1.0}
          : block_t == 64  ? TileCost{0.31, 2.0, 1.5}
          : block_t == 128 ? TileCost{0.50, 2.5, 2.0}
+         : block_t == 192 ? TileCost{0.62, 2.75, 3.0}
                           : TileCost{0.75, 3.0, 4.0};
 }
 constexpr double kLaunchCost = 2.5;
@@ -515,7 +516,8 @@ void consider(int M, int N, int K, Plan* best) {
     const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T>(ks);
     if (per_wave <= 0) continue;
     const int waves = (tiles + per_wave - 1) / per_wave;
-    const bool persistent = BLOCK_T == 256 && ks == 1 && use_persistent<MODE>(M, N, K);
+    bool persistent = false;
+    if constexpr (BLOCK_T >= 192) persistent = ks == 1 && use_persistent<MODE, BLOCK_T>(M, N, K);
     const double per_wave_cost = ((groups + ks - 1) / ks) * c.group + (persistent ? kPersistentBoundary : c.wave) +
                                  (ks > 1 ? c.reduce : 0.0);
     const double cost = kLaunchCost + waves * per_wave_cost;
@@ -531,9 +533,10 @@ void consider(int M, int N, int K, Plan* best) {
 }
 
 // Tokens per tile: the smallest MMA N that covers M up to 128; above that
-// 128- or 256-token tiles, whichever the cost model prefers (256 amortises
-// each converted weight over twice the tokens, 128 wastes fewer rows and
-// fills more SMs at mid M).
+// 128-, 192- or 256-token tiles, whichever the cost model prefers (256
+// amortises each converted weight over the most tokens; 192 and 128 waste
+// fewer rows and fill more SMs at mid M: M=1024 with N=3072 makes 96
+// 256-token tiles for 148 SMs but 144 192-token ones).
 template <int MODE>
 Plan plan_gemm(int M, int N, int K) {
   Plan best;
@@ -555,6 +558,7 @@ Plan plan_gemm(int M, int N, int K) {
     consider<MODE, 128>(M, N, K, &best);
   } else {
     consider<MODE, 128>(M, N, K, &best);
+    consider<MODE, 192>(M, N, K, &best);
     consider<MODE, 256>(M, N, K, &best);
   }
   return best;
@@ -567,12 +571,15 @@ int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales,
   const Plan p = plan_gemm<MODE>(M, N, K);
   if constexpr (MODE != kModeHqq4)
     if (p.small) return launch_gemm_small<MODE>(A, packed, scales, M, N, K, p.ksplit, out, stream);
-  if (p.persistent) return launch_gemm_persistent<MODE>(A, packed, scales, zeros, M, N, K, out, stream);
+  if (p.persistent)
+    return p.block_t == 192 ? launch_gemm_persistent<MODE, 192>(A, packed, scales, zeros, M, N, K, out, stream)
+                            : launch_gemm_persistent<MODE, 256>(A, packed, scales, zeros, M, N, K, out, stream);
   switch (p.block_t) {
     case 16: return launch_gemm<MODE, 16>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 32: return launch_gemm<MODE, 32>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 64: return launch_gemm<MODE, 64>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 128: return launch_gemm<MODE, 128>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+    case 192: return launch_gemm<MODE, 192>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 256: return launch_gemm<MODE, 256>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     default: return BONSAI_ERR_CUDA;  // no plan: the occupancy queries failed
   }
@@ -707,7 +714,7 @@ int bonsai_pack(const int8_t* codes, int64_t N, int64_t K, int mode, void* packe
     pack_b3_kernel<<<grid_for(blocks, 256), 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), N, K);
   } else {
     const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
-    const int grid = grid_for(words / 4, 256);
+    const int grid = grid_for(words / 8, 256);  // two 4-word steps per thread
     if (mode == BONSAI_BINARY)
       pack_kernel<BONSAI_BINARY><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
     else

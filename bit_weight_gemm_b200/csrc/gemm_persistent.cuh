@@ -1,9 +1,10 @@
 // gemm_persistent.cuh - the large-M form of the fused dequantise + GEMM:
-// one persistent CTA per SM walks a list of 128-row x 256-token output tiles.
+// one persistent CTA per SM walks a list of 128-row x BLOCK_T-token output
+// tiles (BLOCK_T = 256, or 192 where 256-token tiles leave a wave part-empty).
 //
 // Same arithmetic, operand layout and stages as lowbit_gemm_kernel (see
 // gemm_tc.cuh): converters turn packed words into exact FP16 products in
-// tensor memory, one thread issues tcgen05.mma (M=128 weight rows, N=256
+// tensor memory, one thread issues tcgen05.mma (M=128 weight rows, N=BLOCK_T
 // tokens, K=16) with A from TMEM and B (activations) from shared memory, and
 // the FP32 sum is rounded once to FP16.  What changes is the tile boundary.
 // With one tile per CTA, each tile paid for its own start (first activation
@@ -32,16 +33,16 @@
 
 namespace bonsai {
 
-template <int MODE>
+template <int MODE, int BLOCK_T>
 struct PersistTile {
-  static constexpr int kBlockT = 256;  // tokens per tile (MMA N)
+  static constexpr int kBlockT = BLOCK_T;  // tokens per tile (MMA N)
   static constexpr int kRows = 128;    // weight rows per tile (MMA M)
   static constexpr bool kB3 = MODE == BONSAI_TERNARY_B3;
   static constexpr bool kHqq = MODE == kModeHqq4;
   static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : (kHqq ? 16 : 8));  // held per group
   static constexpr int kWGroups = kB3 ? kB3BlockGroups : 32 / kWordsPerGroup;  // groups per word stage
   static constexpr int kWRowBytes = kB3 ? kB3BlockBytes : 128;                  // bytes of a row per stage
-  static constexpr int kSliceBytes = kBlockT * 128;     // 256 rows x 64 FP16
+  static constexpr int kSliceBytes = kBlockT * 128;     // BLOCK_T rows x 64 FP16
   static constexpr int kActStageBytes = 2 * kSliceBytes;
   static constexpr int kActStages = 3;
   static constexpr int kWStageBytes = kRows * kWRowBytes;
@@ -51,7 +52,7 @@ struct PersistTile {
   static constexpr int kThreads = 32 * (3 + kConvWarps);
   static constexpr int kACol0 = kBlockT;  // one accumulator, then the converted-weight stages
   static constexpr int kTmemCols = 512;
-  static constexpr int kTStages = (kTmemCols - kACol0) / 64;
+  static constexpr int kTStages = 4;
   static constexpr int kEpiCols = kBlockT / kWarpsPerQuad;  // accumulator columns per converter warp
   static constexpr int kActOff = 0;
   static constexpr int kWOff = kActStages * kActStageBytes;
@@ -66,6 +67,8 @@ struct PersistTile {
   // stage `turn`, and its first group of a tile reuses the stage of the
   // previous tile's group ng - 4 + turn.
   static_assert(kTStages == 4 && kWarpsPerQuad == 4, "stage ownership by turn");
+  static_assert(kACol0 + kTStages * 64 <= kTmemCols, "TMEM budget");
+  static_assert(kBlockT % 64 == 0 && kBlockT <= 256 && kSliceBytes % 1024 == 0, "tile width");
   // Converter warps reading each word stage: all 16, or (4-bit weights, 2
   // groups per stage) the 4 warps of each of its groups.
   static constexpr int kWReaders = 4 * (kWGroups < kWarpsPerQuad ? kWGroups : kWarpsPerQuad);
@@ -79,15 +82,15 @@ struct PersistArgs {
   uint16_t* out;
   int M, N, K;
   int tiles_n;  // 128-row tiles along N; tile tau covers rows (tau % tiles_n) and tokens (tau / tiles_n)
-  int tiles;    // tiles_n x 256-token tiles along M
+  int tiles;    // tiles_n x BLOCK_T-token tiles along M
   uint64_t wait_limit_ns;
 };
 
-template <int MODE>
-__global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
+template <int MODE, int BLOCK_T>
+__global__ void __launch_bounds__(PersistTile<MODE, BLOCK_T>::kThreads, 1)
     lowbit_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmap_act,
                                   const __grid_constant__ CUtensorMap tmap_w, const PersistArgs args) {
-  using T = PersistTile<MODE>;
+  using T = PersistTile<MODE, BLOCK_T>;
   constexpr int AS = T::kActStages, TS = T::kTStages, WS = T::kWStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(PersistTile<MODE>::kThreads, 1)
     };
 
     // Read this warp's share of tile it's accumulator, release it, then round
-    // and store: row n, tokens m0 + c_begin .. +63.
+    // and store: row n, tokens m0 + c_begin .. + kEpiCols - 1.
     auto read_out = [&](int it) -> bool {
       if (!warp_wait(acc_full, it & 1, abort_flag, limit)) return false;
       tc_fence_after_sync();

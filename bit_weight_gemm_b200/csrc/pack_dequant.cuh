@@ -23,66 +23,86 @@ constexpr int kGroup = 128;
 
 __device__ unsigned int g_pack_bad_code = 0;
 
-// Packs 16 ternary codes (one 16-byte load) into one word.  Returns false if
-// any code is outside {-1, 0, +1}.
-__device__ __forceinline__ bool pack_ternary_word(uint4 v, uint32_t& word) {
-  const uint32_t b[4] = {v.x, v.y, v.z, v.w};
-  uint32_t w = 0;
-  bool ok = true;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t code = (b[i >> 2] >> (8 * (i & 3))) & 0xFFu;  // int8 as a byte
-    ok &= (((code + 1u) & 0xFFu) <= 2u);                          // -1, 0, +1 only
-    const int low_bit = 16 * (i & 1) + 14 - 2 * (i >> 1);
-    w |= (code & 3u) << low_bit;  // 0 -> 00, +1 -> 01, -1 (0xFF) -> 11
-  }
-  word = w;
-  return ok;
+// Packing works on four codes (one 32-bit register of int8) at a time.  A
+// byte permute splits the even- and odd-indexed codes (they go to the low and
+// high 16-bit halves of the word); a mask leaves each code's field at bits
+// 8j of its byte j; one multiply then gathers the four fields into the top
+// byte of the product in reverse order (field j at bit 30 - 2j, or 27 - j for
+// one-bit fields), the order the layout wants: the multiplier's other terms
+// land below bit 24 on bits no other term touches, so nothing carries.
+constexpr uint32_t kGather2 = 0x40100401u;  // 2^30 + 2^20 + 2^10 + 1
+constexpr uint32_t kGather1 = 0x08040201u;  // 2^27 + 2^18 + 2^9 + 1
+
+// Nonzero bits for the bytes of x that are not -1, 0 or +1: a valid code is
+// the sign extension of its two low bits, and those bits are not 10.
+__device__ __forceinline__ uint32_t ternary_bad_bytes(uint32_t x) {
+  const uint32_t f = x & 0x03030303u;
+  const uint32_t hi = f & 0x02020202u;
+  return ((f | (hi * 0x7Eu)) ^ x) | (hi & ~(f << 1));
 }
 
-// Packs 32 binary codes (two 16-byte loads) into one word.
-__device__ __forceinline__ bool pack_binary_word(uint4 lo, uint4 hi, uint32_t& word) {
+// Packs 16 ternary codes (one 16-byte load) into one word; `bad` collects
+// nonzero bits if any code is outside {-1, 0, +1}.
+__device__ __forceinline__ uint32_t pack_ternary_word(uint4 v, uint32_t& bad) {
+  const uint32_t e_lo = __byte_perm(v.x, v.y, 0x6420), e_hi = __byte_perm(v.z, v.w, 0x6420);  // codes 0,2,..,14
+  const uint32_t o_lo = __byte_perm(v.x, v.y, 0x7531), o_hi = __byte_perm(v.z, v.w, 0x7531);  // codes 1,3,..,15
+  bad |= ternary_bad_bytes(e_lo) | ternary_bad_bytes(e_hi) | ternary_bad_bytes(o_lo) | ternary_bad_bytes(o_hi);
+  const uint32_t pe_lo = (e_lo & 0x03030303u) * kGather2, pe_hi = (e_hi & 0x03030303u) * kGather2;
+  const uint32_t po_lo = (o_lo & 0x03030303u) * kGather2, po_hi = (o_hi & 0x03030303u) * kGather2;
+  // even codes 0..6 -> bits 15..8, 8..14 -> 7..0; odd codes 1..7 -> 31..24, 9..15 -> 23..16
+  return ((pe_lo >> 16) & 0x0000FF00u) | (pe_hi >> 24) | (po_lo & 0xFF000000u) | ((po_hi >> 8) & 0x00FF0000u);
+}
+
+// Packs 32 binary codes (two 16-byte loads) into one word: the sign bit of
+// each int8 (set for -1) is its bit; `bad` collects nonzero bits for codes
+// other than +1 and -1 (a valid byte is 0x01 with its sign bit spread over
+// bits 1-7).
+__device__ __forceinline__ uint32_t pack_binary_word(uint4 lo, uint4 hi, uint32_t& bad) {
   const uint32_t b[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
   uint32_t w = 0;
-  bool ok = true;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t code = (b[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-    ok &= (code == 0x01u) | (code == 0xFFu);  // +1 or -1
-    const int bit = 16 * (i & 1) + 15 - (i >> 1);
-    w |= (code >> 7) << bit;  // the sign bit of the int8: set for -1
+  for (int g = 0; g < 4; ++g) {  // codes 8g .. 8g+7
+    const uint32_t e = __byte_perm(b[2 * g], b[2 * g + 1], 0x6420);  // codes 8g, 8g+2, 8g+4, 8g+6
+    const uint32_t o = __byte_perm(b[2 * g], b[2 * g + 1], 0x7531);
+    const uint32_t se = (e >> 7) & 0x01010101u, so = (o >> 7) & 0x01010101u;
+    bad |= ((e ^ 0x01010101u) ^ (se * 0xFEu)) | ((o ^ 0x01010101u) ^ (so * 0xFEu));
+    w |= (((se * kGather1) >> 24) & 0xFu) << (12 - 4 * g);  // even codes: bits 15..0
+    w |= (((so * kGather1) >> 24) & 0xFu) << (28 - 4 * g);  // odd codes: bits 31..16
   }
-  word = w;
-  return ok;
+  return w;
 }
 
-// Each thread packs 4 consecutive words and writes them with one 16-byte
-// store.  total_words is a multiple of 4 because K is a multiple of 128.
+// Each thread packs 4 consecutive words per step (one 16-byte store), two
+// steps' loads in flight.  total_words is a multiple of 4 because K is a
+// multiple of 128.
 template <int MODE>
 __global__ void __launch_bounds__(256) pack_kernel(const int8_t* __restrict__ codes, uint32_t* __restrict__ packed,
                                                    int64_t total_words) {
   constexpr int kPerWord = MODE == BONSAI_BINARY ? 32 : 16;
+  constexpr int kLoads = kPerWord / 4;  // 16-byte loads per 4 words
   const int64_t quads = total_words / 4;
-  bool ok = true;
-  for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < quads; q += (int64_t)gridDim.x * blockDim.x) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  uint32_t bad = 0;
+  for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < quads; q += 2 * stride) {
+    const bool two = q + stride < quads;
+    uint4 v[2][kLoads];
     const uint4* src = reinterpret_cast<const uint4*>(codes + q * 4 * kPerWord);
-    uint32_t w[4];
-    if (MODE == BONSAI_BINARY) {
-      uint4 v[8];
+    const uint4* src2 = reinterpret_cast<const uint4*>(codes + (two ? q + stride : q) * 4 * kPerWord);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = __ldg(src + i);
+    for (int i = 0; i < kLoads; ++i) v[0][i] = __ldg(src + i);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ok &= pack_binary_word(v[2 * i], v[2 * i + 1], w[i]);
-    } else {
-      uint4 v[4];
+    for (int i = 0; i < kLoads; ++i) v[1][i] = __ldg(src2 + i);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = __ldg(src + i);
+    for (int h = 0; h < 2; ++h) {
+      uint32_t w[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ok &= pack_ternary_word(v[i], w[i]);
+      for (int i = 0; i < 4; ++i)
+        w[i] = MODE == BONSAI_BINARY ? pack_binary_word(v[h][2 * i], v[h][2 * i + 1], bad)
+                                     : pack_ternary_word(v[h][i], bad);
+      if (h == 0 || two) reinterpret_cast<uint4*>(packed)[h == 0 ? q : q + stride] = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    reinterpret_cast<uint4*>(packed)[q] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  if (!__all_sync(0xffffffffu, ok) && lane_id() == 0) atomicOr(&g_pack_bad_code, 1u);
+  if (!__all_sync(0xffffffffu, bad == 0) && lane_id() == 0) atomicOr(&g_pack_bad_code, 1u);
 }
 
 // Exact dequantisation.  Each thread expands one packed word: 16 (ternary)

@@ -198,8 +198,9 @@ def _sms():
 def test_plans_cover_every_form():
     big = bw.gemm_plan(4608, 9216, 3072, "ternary")  # persistent: one CTA per SM walks 1296 tiles
     assert big == {"block_t": 256, "ksplit": 1, "ctas": _sms(), "tiles": 72 * 18}
-    one_wave = bw.gemm_plan(1024, 3072, 3072, "binary")  # 96 tiles: one CTA (or cluster) each
-    assert one_wave["tiles"] == 24 * 4 and one_wave["ctas"] == one_wave["tiles"] * one_wave["ksplit"]
+    one_wave = bw.gemm_plan(1024, 3072, 3072, "binary")  # 144 192-token tiles: one CTA each, one wave
+    assert one_wave["block_t"] == 192 and one_wave["tiles"] == 24 * 6
+    assert one_wave["ctas"] == one_wave["tiles"] * one_wave["ksplit"]
     for M, N, K in [(16, 3072, 9216), (16, 9216, 3072), (16, 256, 4096), (40, 384, 2048)]:
         p = bw.gemm_plan(M, N, K, "ternary")
         assert 1 < p["ksplit"] <= 8 and p["ctas"] == p["tiles"] * p["ksplit"], (M, N, K, p)
@@ -238,6 +239,28 @@ LARGE_M_SHAPES = [
     ("ternary", 1357, 3880, 640, False),
     ("binary", 600, 6376, 512, False),
 ]
+
+
+# 192-token tiles, where 256-token ones would leave SMs idle: one wave of
+# one-tile CTAs (M=1024 / 1000 with N=3072 / 3000: 144 tiles) and the
+# persistent kernel (M=2048 with N=3072: 264 tiles); ragged M and N.
+TILE192_SHAPES = [
+    ("binary", 1024, 3072, 3072, False),
+    ("ternary", 1000, 3000, 1152, False),
+    ("ternary_b3", 1000, 3000, 1152, False),
+    ("ternary", 2048, 3072, 2048, True),
+    ("ternary_b3", 2000, 3050, 2048, True),
+    ("binary", 2048, 3072, 2048, True),
+]
+
+
+@pytest.mark.parametrize("mode,M,N,K,persistent", TILE192_SHAPES)
+def test_gemm_192_token_tiles(oracle_mod, mode, M, N, K, persistent):
+    plan = bw.gemm_plan(M, N, K, mode)
+    assert plan["block_t"] == 192 and plan["ksplit"] == 1, plan
+    assert (plan["ctas"] < plan["tiles"]) == persistent, plan
+    got, ref, absacc = _gemm_case(oracle_mod, mode, M, N, K, seed=M + 5 * N + 3 * K)
+    assert_gemm_close(oracle_mod, got, ref, absacc, f"{mode} {M}x{N}x{K}")
 
 
 @pytest.mark.parametrize("mode,M,N,K,persistent", LARGE_M_SHAPES)
@@ -536,7 +559,8 @@ def test_hqq4_pack_reports_bad_values():
     assert e.value.status == 4
 
 
-@pytest.mark.parametrize("M,N,K", SMALL_SHAPES + [(1357, 3880, 512), (700, 1000, 640), (16, 3072, 12288)])
+@pytest.mark.parametrize("M,N,K", SMALL_SHAPES + [(1357, 3880, 512), (700, 1000, 640), (16, 3072, 12288),
+                                   (1000, 3000, 1152), (2048, 3072, 2048)])
 def test_hqq4_gemm_full(oracle_mod, M, N, K):
     d = workloads.make_hqq4(M, N, K, seed=M + 5 * N + K)
     packed, s, z, A = _hqq4_inputs(d)
