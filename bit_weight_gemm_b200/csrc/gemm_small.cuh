@@ -25,8 +25,10 @@
 //    stage reads it back before converting its next group into the stage,
 //    adding s_g * D_g into registers.
 //  - Equal work per CTA in one wave: the launch is tiles x ksplit CTAs, every
-//    CTA holding the same number of 128-wide groups (at most 18), with ksplit
-//    the largest split whose clusters all fit on the GPU at once.  The ksplit
+//    CTA holding the same number of 128-wide groups (at most 24).  With no
+//    split on at most half the SMs, the next launch's CTAs start on the other
+//    half while this one runs; otherwise ksplit is the largest split (up to
+//    5) whose clusters all fit on the GPU at once.  The ksplit
 //    CTAs of a tile form a cluster: ranks 1.. push their FP32 partial tile
 //    into rank 0's shared memory with st.async, counted on rank 0's mbarrier,
 //    and leave; rank 0 adds the partials in rank order (deterministic),
@@ -60,7 +62,7 @@ struct SmallTile {
   static constexpr int kWRowBytes = kB3 ? kB3BlockBytes : 128;
   static constexpr int kWStageBytes = kRows * kWRowBytes;
   static constexpr int kGroupAlign = kB3 ? kB3BlockGroups : 1;
-  static constexpr int kMaxGroups = 18;  // groups per CTA: the whole slice stays in shared memory
+  static constexpr int kMaxGroups = 24;  // groups per CTA: the whole slice stays in shared memory
   static constexpr int kWStages = (kMaxGroups + kWGroups - 1) / kWGroups;
   static constexpr int kSliceBytes = kBlockT * 128;         // 16 rows x 64 FP16, one SW128 K slice
   static constexpr int kActGroupBytes = 2 * kSliceBytes;    // one group's activations
@@ -70,7 +72,7 @@ struct SmallTile {
   static constexpr int kTmemCols = 512;
   static constexpr int kAccCol0 = 64 * kTurns;  // stage t: weights at 64t, accumulator at kAccCol0 + 16t
   static constexpr int kGranules = kBlockT * kRows / 4;  // 4 consecutive rows of one token
-  static constexpr int kMaxSplit = 8;                     // CTAs per cluster
+  static constexpr int kMaxSplit = 5;                     // CTAs per cluster
   static constexpr int kRecvBytes = (kMaxSplit - 1) * kGranules * 16;  // rank 0 receives the other ranks' partials
   static constexpr int kWOff = 0;
   static constexpr int kActOff = kWOff + kWStages * kWStageBytes;

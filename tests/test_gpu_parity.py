@@ -201,9 +201,11 @@ def test_plans_cover_every_form():
     one_wave = bw.gemm_plan(1024, 3072, 3072, "binary")  # 144 192-token tiles: one CTA each, one wave
     assert one_wave["block_t"] == 192 and one_wave["tiles"] == 24 * 6
     assert one_wave["ctas"] == one_wave["tiles"] * one_wave["ksplit"]
-    for M, N, K in [(16, 3072, 9216), (16, 9216, 3072), (16, 256, 4096), (40, 384, 2048)]:
+    for M, N, K in [(16, 3072, 9216), (16, 256, 4096), (40, 384, 2048)]:
         p = bw.gemm_plan(M, N, K, "ternary")
         assert 1 < p["ksplit"] <= 8 and p["ctas"] == p["tiles"] * p["ksplit"], (M, N, K, p)
+    # 72 tiles of 24 groups at 16 tokens: no split, on half the SMs (the next launch starts beside it)
+    assert bw.gemm_plan(16, 9216, 3072, "ternary") == {"block_t": 16, "ksplit": 1, "ctas": 72, "tiles": 72}
     assert bw.gemm_plan(0, 8, 128, "binary") == {"block_t": 0, "ksplit": 0, "ctas": 0, "tiles": 0}
 
 
