@@ -502,16 +502,25 @@ def time_formats(torch, bw, args, dist, peaks, peaks_kind):
                     "us_per_launch": t * 1e6, "packed_bytes": packed_weight_bytes(p.mode, p.N, p.K),
                     "int2_packed_bytes": packed_weight_bytes("ternary", p.N, p.K),
                     "plan": bw.gemm_plan(p.M, p.N, p.K, p.mode)})
-    # 4-bit group-affine weights (the text encoder's format) on the headline shape
-    p = WORKLOAD
+    # 4-bit group-affine weights (the text encoder's format) on the headline shape and at M=16
+    for p, unit in ((WORKLOAD, "TFLOP/s"), (SMALL[0], "GB/s")):
+        out.append(time_hqq4(torch, bw, args, p, unit))
+    return out
+
+
+def time_hqq4(torch, bw, args, p, unit):
+    """The 4-bit group-affine GEMM on problem p's shape: TFLOP/s, or GB/s of
+    its algorithmic bytes (packed 4-bit words, FP16 scales and zeros per 64,
+    activations in, output out)."""
     d = workloads.make_hqq4(1, p.N, p.K, seed=p.seed)
     packed = bw.hqq4_pack(torch.from_numpy(d["q"]).cuda())
     s = torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda()
     z = torch.from_numpy(d["zeros"].view(np.int16)).view(torch.float16).cuda()
     rng = np.random.default_rng(p.seed)
+    nsets = args.sets if unit == "TFLOP/s" else 32  # above L2 either way
     sets = [(torch.from_numpy(workloads.activations(rng, p.M, p.K).view(np.int16)).view(torch.float16).cuda(),
              packed.clone(), s.clone(), z.clone(), torch.empty((p.M, p.N), dtype=torch.float16, device="cuda"))
-            for _ in range(args.sets)]
+            for _ in range(nsets)]
 
     def launch(i):
         A, pk, sc, zc, o = sets[i % len(sets)]
@@ -535,10 +544,11 @@ def time_formats(torch, bw, args, dist, peaks, peaks_kind):
     torch.cuda.synchronize()
     t = e0.elapsed_time(e1) / 1e3 / steps
     del graph, sets
-    out.append({"workload": "4-bit group-affine " + p.name, "mode": "hqq4", "M": p.M, "N": p.N, "K": p.K,
-                "value": flops(p) / t / 1e12, "unit": "TFLOP/s", "us_per_launch": t * 1e6,
-                "packed_bytes": p.N * p.K // 2, "plan": bw.gemm_plan(p.M, p.N, p.K, "hqq4")})
-    return out
+    nbytes = p.N * p.K // 2 + 4 * p.N * (p.K // 64) + 2 * p.M * p.K + 2 * p.M * p.N
+    return {"workload": "4-bit group-affine " + p.name, "mode": "hqq4", "M": p.M, "N": p.N, "K": p.K,
+            "value": flops(p) / t / 1e12 if unit == "TFLOP/s" else nbytes / t / 1e9, "unit": unit,
+            "us_per_launch": t * 1e6, "packed_bytes": p.N * p.K // 2, "algorithmic_bytes": nbytes,
+            "plan": bw.gemm_plan(p.M, p.N, p.K, "hqq4")}
 
 
 LAYER_SHAPES = ((18432, 3072, "single-stream fused QKV + MLP-up"), (3072, 12288, "single-stream out"))

@@ -106,10 +106,31 @@ __global__ void __launch_bounds__(256) pack_kernel(const int8_t* __restrict__ co
 }
 
 // Exact dequantisation.  Each thread expands one packed word: 16 (ternary)
-// or 32 (binary) FP16 weights, 32 or 64 contiguous bytes.  The code becomes
-// an exact FP16 t (ternary: the shifted field is 2t, halved exactly; binary:
-// the sign bit over 1.0) and one IEEE FP16 multiply by the scale gives
-// t * s with the product's sign-of-zero and NaN rules.
+// or 32 (binary) FP16 weights, 32 or 64 contiguous bytes.  The code becomes an exact FP16 t (ternary: the shifted field is 2t,
+// halved exactly; binary: the sign bit over 1.0) and one IEEE FP16 multiply
+// by the scale gives t * s with the product's sign-of-zero and NaN rules.
+template <int MODE>
+__device__ __forceinline__ void dequant_word(uint32_t word, uint32_t s2, uint16_t* dst) {
+  constexpr int kPerWord = MODE == BONSAI_BINARY ? 32 : 16;
+  uint32_t v[kPerWord / 2];
+  if (MODE == BONSAI_BINARY) {
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const uint32_t t = ((word << p) & 0x80008000u) | 0x3C003C00u;  // +-1.0 pair
+      v[p] = hmul2_bits(t, s2);
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const uint32_t two_t = (word << (2 * p)) & 0xC000C000u;  // {0, +-2.0} pair (-0 for the non-code)
+      v[p] = hmul2_bits(hmul2_bits(two_t, 0x38003800u), s2);  // * 0.5 (exact), then * s
+    }
+  }
+  uint4* out = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < kPerWord / 8; ++i) out[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict__ packed,
                                                       const uint16_t* __restrict__ scales, uint16_t* __restrict__ w,
@@ -120,28 +141,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
   const int64_t total = N * words_per_row;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t n = idx / words_per_row;
-    const int64_t j = idx - n * words_per_row;
-    const uint32_t word = __ldg(packed + idx);
+    const int64_t n = idx / words_per_row, j = idx - n * words_per_row;
     const uint32_t s = __ldg(scales + n * groups + (j * kPerWord) / kGroup);
-    const uint32_t s2 = s | (s << 16);
-    uint32_t v[kPerWord / 2];
-    if (MODE == BONSAI_BINARY) {
-#pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        const uint32_t t = ((word << p) & 0x80008000u) | 0x3C003C00u;  // +-1.0 pair
-        v[p] = hmul2_bits(t, s2);
-      }
-    } else {
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const uint32_t two_t = (word << (2 * p)) & 0xC000C000u;  // {0, +-2.0} pair (-0 for the non-code)
-        v[p] = hmul2_bits(hmul2_bits(two_t, 0x38003800u), s2);  // * 0.5 (exact), then * s
-      }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(w + n * K + j * kPerWord);
-#pragma unroll
-    for (int i = 0; i < kPerWord / 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    dequant_word<MODE>(__ldg(packed + idx), s | (s << 16), w + n * K + j * kPerWord);
   }
 }
 
