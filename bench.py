@@ -58,7 +58,7 @@ def parse_args():
     ap.add_argument("--case", default=None,
                     help="run one configuration --launches times, untimed (the command the committed ncu summaries "
                          "profile): MODE:M:N:K for the GEMM (MODE binary, ternary, ternary_b3 or hqq4), "
-                         "pack-MODE:N:K or dequant-MODE:N:K")
+                         "pack-MODE:N:K, dequant-MODE:N:K, or batch-MODE:M:N:K:L for L layers in one batch call")
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--m-sweep", action="store_true",
                     help="time the GEMM over M = 16..4608 on the stack's five layer shapes and print one JSON line")
@@ -372,9 +372,10 @@ def run_bonsai(args):
             e2e = time_e2e(torch, bw, p, min(args.steps, 50), 3, dist)
         result["e2e"] = e2e
 
-    small = None
+    small = small_batch = None
     if not args.no_extras or args.small_only:
         small = [time_small(torch, bw, sp, args, dist, peaks, peaks_kind) for sp in SMALL]
+        small_batch = time_small_batch(torch, bw, args, dist, peaks, peaks_kind)
     stack = None
     if not args.no_extras and not args.small_only:
         stack = [time_stack(torch, bw, m, "ternary", 20, 3) for m in (4608, 1024)]
@@ -396,7 +397,7 @@ def run_bonsai(args):
         dist.barrier()
     if rank == 0:
         if args.small_only:
-            print(json.dumps({"small_m": small}), flush=True)
+            print(json.dumps({"small_m": small, "small_m_batch": small_batch}), flush=True)
         else:
             traffic = ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}")
             line = {
@@ -417,6 +418,7 @@ def run_bonsai(args):
                 "e2e": result["e2e"],
                 "cpu_baseline": cpu,
                 "small_m": small,
+                "small_m_batch": small_batch,
                 "stack": stack,
                 "layers": layers,
                 "formats": formats,
@@ -483,6 +485,77 @@ def time_small(torch, bw, p, args, dist, peaks, peaks_kind):
                          "frac": achieved / peak, "traffic": ncu_traffic(f"{p.mode}_M{p.M}_N{p.N}_K{p.K}"),
                          "algorithmic_bytes_per_launch": nbytes, "peak_source": f"{peaks_kind} hbm copy"},
             "gpu_launches": steps}
+
+
+BATCH_LAYERS = 80  # one denoise step's worth of linears per call
+
+
+def time_small_batch(torch, bw, args, dist, peaks, peaks_kind):
+    """The bandwidth-bound regime with many layers per call: 80 independent
+    16-token GEMMs in one bonsai_lowbit_gemm_batch call (one persistent
+    launch), each layer with its own buffers (633-752 MB in all, 5-6x L2, so
+    every weight byte comes from HBM).  Three batches: 80 MLP-down layers
+    (3072x9216), 80 fused-QKV layers (9216x3072), and the 80 linears of one
+    denoise step.  GB/s of algorithmic bytes (packed weights, scales,
+    activations, outputs of all layers) per call; the call is replayed from a
+    CUDA graph and timed with CUDA events on the replay stream."""
+    out = []
+    step_layers = [(n, k) for _, n, k in workloads.mmdit_stack_layers()]
+    cases = [("ternary MLP-down M=16 x 80 layers", [(SMALL[0].N, SMALL[0].K)] * BATCH_LAYERS, SMALL[0].seed),
+             ("ternary fused QKV M=16 x 80 layers", [(SMALL[1].N, SMALL[1].K)] * BATCH_LAYERS, SMALL[1].seed),
+             ("ternary denoise-step linears M=16 (80 layers)", step_layers, 3000)]
+    for name, shapes, seed in cases:
+        base = {}
+        probs, nbytes = [], 0
+        for j, (n, k) in enumerate(shapes):
+            p = workloads.Problem(name, "ternary", 16, n, k, seed + j)
+            if (n, k) not in base:
+                d = workloads.make(p)
+                base[(n, k)] = (torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).cuda(),
+                                bw.pack(torch.from_numpy(d["codes"]).cuda(), "ternary"),
+                                torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda())
+            A, packed, sc = (t.clone() for t in base[(n, k)])  # own buffers: every layer reads its own bytes
+            probs.append((A, packed, sc))
+            nbytes += algorithmic_bytes(p)
+        outs = [torch.empty((16, n), dtype=torch.float16, device="cuda") for n, _ in shapes]
+        torch.cuda.synchronize()
+
+        def call():
+            bw.lowbit_gemm_batch(probs, "ternary", outs=outs)
+
+        for _ in range(max(args.warmup, 3)):
+            call()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        graph.replay()
+        steps = 50
+        stream = torch.cuda.current_stream()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        del graph
+        per_call = max_over_ranks(torch, start.elapsed_time(end) / 1e3, dist) / steps
+        achieved = nbytes / per_call / 1e9
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        flop = sum(2 * 16 * n * k for n, k in shapes)
+        out.append({"workload": name, "M": 16, "layers": len(shapes), "value": achieved, "unit": "GB/s",
+                    "us_per_call": per_call * 1e6, "us_per_layer": per_call * 1e6 / len(shapes),
+                    "tflops": flop / per_call / 1e12, "api": "bonsai_lowbit_gemm_batch, one call per step",
+                    "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                                 "frac": achieved / peak, "traffic": ncu_traffic(f"batch_{name}"),
+                                 "algorithmic_bytes_per_call": nbytes, "peak_source": f"{peaks_kind} hbm copy"},
+                    "gpu_launches": steps})
+        del probs, outs, base
+    return out
 
 
 def time_formats(torch, bw, args, dist, peaks, peaks_kind):
@@ -804,10 +877,26 @@ def run_case(args):
     torch.cuda.set_device(0)
     import bit_weight_gemm_b200 as bw
 
-    op, _, rest = args.case.rpartition("-") if args.case.split(":")[0].startswith(("pack-", "dequant-")) else \
-        ("gemm", "", args.case)
+    op, _, rest = args.case.rpartition("-") if args.case.split(":")[0].startswith(("pack-", "dequant-", "batch-")) \
+        else ("gemm", "", args.case)
     fields = rest.split(":")
     mode = fields[0]
+    if op == "batch":
+        # batch-MODE:M:N:K:L - L layers of one shape (own buffers each) in one bonsai_lowbit_gemm_batch call
+        M, N, K, L = (int(x) for x in fields[1:5])
+        d = workloads.make(mode=mode, M=M, N=N, K=K, seed=7)
+        base = (torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).cuda(),
+                bw.pack(torch.from_numpy(d["codes"]).cuda(), mode),
+                torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda())
+        probs = [tuple(t.clone() for t in base) for _ in range(L)]
+        outs = [torch.empty((M, N), dtype=torch.float16, device="cuda") for _ in range(L)]
+        torch.cuda.synchronize()
+        for _ in range(args.launches):
+            bw.lowbit_gemm_batch(probs, mode, outs=outs)
+        torch.cuda.synchronize()
+        assert bw.get_device_error() == 0
+        print(json.dumps({"case": args.case, "launches": args.launches}), flush=True)
+        return 0
     if op == "gemm":
         M, N, K = (int(x) for x in fields[1:4])
     else:

@@ -26,6 +26,13 @@ _lib = None
 # Every function the C header declares, with its ctypes signature.
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
+
+
+class GemmProblem(ctypes.Structure):
+    """bonsai_gemm_problem: one GEMM of a bonsai_lowbit_gemm_batch call."""
+    _fields_ = [("A", _P), ("packed", _P), ("scales", _P), ("out", _P), ("M", _I64), ("N", _I64), ("K", _I64)]
+
+
 SIGNATURES = {
     "bonsai_packed_bytes": (ctypes.c_size_t, [_I64, _I64, ctypes.c_int]),
     "bonsai_scale_bytes": (ctypes.c_size_t, [_I64, _I64]),
@@ -37,6 +44,7 @@ SIGNATURES = {
     "bonsai_hqq4_dequant": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
     "bonsai_hqq4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "bonsai_lowbit_gemm_host": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P]),
+    "bonsai_lowbit_gemm_batch": (ctypes.c_int, [ctypes.POINTER(GemmProblem), ctypes.c_int, ctypes.c_int, _P]),
     "bonsai_gemm_plan": (ctypes.c_int, [_I64, _I64, _I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
                                         ctypes.POINTER(ctypes.c_int)]),
@@ -153,6 +161,29 @@ def lowbit_gemm(A: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, mod
                                     _dev(scales, "scales", torch.float16), M, N, K, m,
                                     _dev(out, "out", torch.float16), _stream()), "bonsai_lowbit_gemm")
     return out
+
+
+def lowbit_gemm_batch(problems, mode, outs=None) -> list:
+    """Independent GEMMs in one call: problems is a sequence of (A [M,K],
+    packed, scales) device tensors of one mode; returns their FP16 outputs
+    [M,N] (or fills `outs`).  Problems of up to 16 tokens share persistent
+    launches; larger ones are launched one by one."""
+    m = _mode(mode)
+    n = len(problems)
+    arr = (GemmProblem * max(n, 1))()
+    result = []
+    for i, (A, packed, scales) in enumerate(problems):
+        M, K = A.shape
+        N = packed.shape[0]
+        out = outs[i] if outs is not None else torch.empty((M, N), dtype=torch.float16, device=A.device)
+        if tuple(out.shape) != (M, N):
+            raise ValueError(f"outs[{i}] must be [{M}, {N}]")
+        arr[i] = GemmProblem(_dev(A, "A", torch.float16).value, _dev(packed, "packed").value,
+                             _dev(scales, "scales", torch.float16).value, _dev(out, "out", torch.float16).value,
+                             M, N, K)
+        result.append(out)
+    _check(lib().bonsai_lowbit_gemm_batch(arr, n, m, _stream()), "bonsai_lowbit_gemm_batch")
+    return result
 
 
 def _host(t: torch.Tensor, name: str) -> ctypes.c_void_p:

@@ -1,15 +1,18 @@
 // bonsai.cu - the C ABI declared in include/bonsai.h: argument checks, tensor
-// maps, kernel selection (the planner) and launches, and the host-buffer
-// pipeline.  All arithmetic runs in the kernels of pack_dequant.cuh,
-// gemm_tc.cuh and gemm_persistent.cuh.
+// maps, kernel selection (the planner) and launches, the batched small-M
+// launches, and the host-buffer pipeline.  All arithmetic runs in the kernels
+// of pack_dequant.cuh, gemm_tc.cuh, gemm_persistent.cuh, gemm_small.cuh and
+// gemm_batch.cuh.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "bonsai.h"
+#include "gemm_batch.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_small.cuh"
 #include "gemm_tc.cuh"
@@ -479,6 +482,67 @@ int launch_gemm_small(const uint16_t* A, const void* packed, const uint16_t* sca
   return launch_status();
 }
 
+// ------------------------------------------------- batched small M --
+// One persistent launch over `count` problems of up to 16 tokens
+// (gemm_batch.cuh): their 128-row tiles form one unit list, cut into one
+// contiguous range per CTA with nearly equal numbers of K groups.
+template <int MODE>
+int launch_gemm_batch(const bonsai_gemm_problem* const* probs, int count, cudaStream_t stream) {
+  using T = BatchTile<MODE>;
+  if (count < 1 || count > kBatchMaxLayers) return BONSAI_ERR_INVALID_ARG;
+  if (smem_opt_in<lowbit_gemm_batch_kernel<MODE>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
+  static thread_local BatchParams params;  // 28 KB: kept off the stack
+  int units = 0;
+  int64_t total = 0;  // K groups of all units
+  for (int i = 0; i < count; ++i) {
+    const bonsai_gemm_problem& q = *probs[i];
+    const int M = static_cast<int>(q.M), N = static_cast<int>(q.N), K = static_cast<int>(q.K);
+    if (!make_map(&params.act[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q.A, K, M, 64, T::kBlockT,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+      return BONSAI_ERR_CUDA;
+    if (!make_weight_map(&params.w[i], q.packed, N, K, MODE)) return BONSAI_ERR_CUDA;
+    params.layer[i] = BatchLayer{q.scales, q.out, M, N, K, units};
+    const int tiles = (N + T::kRows - 1) / T::kRows;
+    units += tiles;
+    total += static_cast<int64_t>(tiles) * (K / kGroup);
+  }
+  params.count = count;
+  params.units = units;
+  params.wait_limit_ns = kDefaultWaitLimitNs;
+  int ctas = sm_count();
+  if (ctas > kBatchMaxCtas) ctas = kBatchMaxCtas;
+  if (ctas > units) ctas = units;
+  // Boundary c: units go to the earlier CTA while at least half of a unit's
+  // groups lie before c * total / ctas.
+  params.cta_unit0[0] = 0;
+  int u = 0, li = 0;
+  int64_t before = 0;  // groups of units 0 .. u-1
+  for (int c = 1; c < ctas; ++c) {
+    const int64_t target = total * c / ctas;
+    while (u < units) {
+      while (li + 1 < count && params.layer[li + 1].unit0 <= u) ++li;
+      const int g = params.layer[li].K / kGroup;
+      if (2 * (before + g) > 2 * target + g) break;
+      before += g;
+      ++u;
+    }
+    params.cta_unit0[c] = u;
+  }
+  params.cta_unit0[ctas] = units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(T::kThreads);
+  cfg.dynamicSmemBytes = T::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, lowbit_gemm_batch_kernel<MODE>, params) != cudaSuccess) return BONSAI_ERR_CUDA;
+  return launch_status();
+}
+
 // ------------------------------------------------------------- planning --
 // Launch costs in microseconds, measured on a B200 with an M sweep of single
 // launches (16..4608 tokens on the MMDiT layer shapes, clocks under the power
@@ -801,6 +865,61 @@ int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const ui
   if (mode == BONSAI_TERNARY_B3)
     return gemm_host_pipelined<BONSAI_TERNARY_B3>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
   return gemm_host_pipelined<BONSAI_TERNARY_INT2>(A_host, packed, scales, M, N, K, out_host, A_dev, out_dev, st);
+}
+
+int bonsai_lowbit_gemm_batch(const bonsai_gemm_problem* problems, int count, int mode, void* stream) {
+  if (!valid_mode(mode)) return BONSAI_ERR_INVALID_ARG;
+  if (count < 0 || (count > 0 && !problems)) return BONSAI_ERR_INVALID_ARG;
+  bool any = false;
+  for (int i = 0; i < count; ++i) {
+    const bonsai_gemm_problem& q = problems[i];
+    int rc = check_shape(q.M, q.N, q.K);
+    if (rc != BONSAI_OK) return rc;
+    if (q.M == 0 || q.N == 0) continue;
+    if (!q.out) return BONSAI_ERR_INVALID_ARG;
+    if (!aligned16(q.out)) return BONSAI_ERR_ALIGN;
+    if (q.K > 0) {
+      if (!q.A || !q.packed || !q.scales) return BONSAI_ERR_INVALID_ARG;
+      if (!aligned16(q.A) || !aligned16(q.packed) || !aligned16(q.scales)) return BONSAI_ERR_ALIGN;
+    }
+    any = true;
+  }
+  if (!any) return BONSAI_OK;
+  int rc = check_device();
+  if (rc != BONSAI_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<const bonsai_gemm_problem*> small;
+  for (int i = 0; i < count; ++i) {
+    const bonsai_gemm_problem& q = problems[i];
+    if (q.M == 0 || q.N == 0) continue;
+    if (q.K == 0) {  // empty sums
+      if (cudaMemsetAsync(q.out, 0, static_cast<size_t>(q.M) * q.N * 2, st) != cudaSuccess) return BONSAI_ERR_CUDA;
+    } else if (q.M <= 16) {
+      small.push_back(&q);
+    }
+  }
+  // Launches of nearly equal numbers of problems, at most kBatchMaxLayers each.
+  const int n_small = static_cast<int>(small.size());
+  const int launches = (n_small + kBatchMaxLayers - 1) / kBatchMaxLayers;
+  for (int l = 0; l < launches; ++l) {
+    const int b = static_cast<int>(static_cast<int64_t>(n_small) * l / launches);
+    const int e = static_cast<int>(static_cast<int64_t>(n_small) * (l + 1) / launches);
+    rc = mode == BONSAI_BINARY      ? launch_gemm_batch<BONSAI_BINARY>(small.data() + b, e - b, st)
+         : mode == BONSAI_TERNARY_B3 ? launch_gemm_batch<BONSAI_TERNARY_B3>(small.data() + b, e - b, st)
+                                     : launch_gemm_batch<BONSAI_TERNARY_INT2>(small.data() + b, e - b, st);
+    if (rc != BONSAI_OK) return rc;
+  }
+  for (int i = 0; i < count; ++i) {
+    const bonsai_gemm_problem& q = problems[i];
+    if (q.M <= 16 || q.N == 0 || q.K == 0) continue;
+    const int m = static_cast<int>(q.M), n = static_cast<int>(q.N), k = static_cast<int>(q.K);
+    rc = mode == BONSAI_BINARY ? dispatch_gemm<BONSAI_BINARY>(q.A, q.packed, q.scales, nullptr, m, n, k, q.out, st)
+         : mode == BONSAI_TERNARY_B3
+             ? dispatch_gemm<BONSAI_TERNARY_B3>(q.A, q.packed, q.scales, nullptr, m, n, k, q.out, st)
+             : dispatch_gemm<BONSAI_TERNARY_INT2>(q.A, q.packed, q.scales, nullptr, m, n, k, q.out, st);
+    if (rc != BONSAI_OK) return rc;
+  }
+  return BONSAI_OK;
 }
 
 // ------------------------------------------ 4-bit group-affine weights --

@@ -159,6 +159,12 @@ struct GemmTile {
   static_assert(kMmaThreads == 1 || (kTStages - kWarpsPerQuad) % 2 == 0, "same MMA warp for groups i-q-TS, i-2TS");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(kActStages >= 2, "activation ring depth");
+  // Parity waits are unambiguous only for a waiter that meets every phase of
+  // a barrier, or whose skipped phases are known complete.  Two MMA warps take
+  // alternate groups: with an even number of stages each of them (and each of
+  // the two activation producers) keeps to its own stages.  With one MMA warp
+  // the stages are released in order, which covers the producers' skips.
+  static_assert(kMmaThreads == 1 || kActStages % 2 == 0, "alternate groups keep to their own stages");
   static_assert(BLOCK_T * kRows * 2 <= kActStages * kActStageBytes, "output tile fits the act ring");
   static_assert(kRows * BLOCK_T * 4 <= kActStages * kActStageBytes, "partial fits the act ring");
 };

@@ -155,6 +155,40 @@ int bonsai_lowbit_gemm_host(const uint16_t* A_host, const void* packed, const ui
                             int64_t N, int64_t K, int mode, uint16_t* out_host, uint16_t* A_dev,
                             uint16_t* out_dev, void* stream);
 
+/* One problem of bonsai_lowbit_gemm_batch: out = A * w^T for an [N,K]
+ * weight, with the operands, layouts and rules of bonsai_lowbit_gemm. */
+typedef struct {
+  const uint16_t* A;      /* FP16 [M,K], device */
+  const void* packed;     /* packed [N,K] weight (bonsai_pack), device */
+  const uint16_t* scales; /* FP16 [N,K/128], device */
+  uint16_t* out;          /* FP16 [M,N], device */
+  int64_t M, N, K;
+} bonsai_gemm_problem;
+
+/* Several independent low-bit GEMMs in one call, all of one weight mode
+ * (no counterpart of its own on the pages; it serves their bandwidth-bound
+ * case: at a few tokens a quantised linear is a stream of its packed
+ * weights, and the weight bytes of the transformer's linears per denoising
+ * step set its speed, "Introducing 1-bit and Ternary Bonsai Image 4B: Image
+ * Generation for Local Devices", section "端侧约束：为什么 diffusion
+ * transformer 是唯一值得压缩的部分").
+ * Problems with M <= 16 run together in persistent launches of up to 96
+ * problems each: one CTA per SM walks the 128-row weight tiles of all of
+ * them, so the weight stream does not stop between problems for a launch,
+ * a dependency release and a tail of its own.  Problems with M > 16 are
+ * launched one by one, as bonsai_lowbit_gemm launches them.  Each result
+ * is the one bonsai_lowbit_gemm gives up to the order of the FP32 sums (the
+ * same accuracy).
+ * problems: HOST array of `count` entries, read during the call only.
+ * Independence: no problem's out may overlap any A, packed, scales or out
+ * of the batch; the order of the launches is unspecified.
+ * Stream order: as for bonsai_lowbit_gemm (the weights of the first problems
+ * may be read while the kernel enqueued just before still runs).
+ * Errors: every problem is checked before anything is launched and the
+ * first error found is returned; BONSAI_ERR_INVALID_ARG also for count < 0
+ * or a NULL problems with count > 0. */
+int bonsai_lowbit_gemm_batch(const bonsai_gemm_problem* problems, int count, int mode, void* stream);
+
 /* ------------------------------------------ 4-bit group-affine weights --
  * The pages name "4-bit HQQ" for the text encoder ("Cómo Bonsai Ternary 4B
  * revoluciona la difusión texto-imagen", section "Arquitectura de despliegue

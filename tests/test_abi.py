@@ -30,6 +30,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for required in ["bonsai_pack", "bonsai_dequant", "bonsai_lowbit_gemm", "bonsai_lowbit_gemm_host",
+                     "bonsai_lowbit_gemm_batch",
                      "bonsai_get_device_error",
                      "bonsai_status_string", "bonsai_packed_bytes", "bonsai_scale_bytes"]:
         assert required in names
@@ -103,6 +104,29 @@ def test_argument_errors_before_any_device_work(lib):
     assert lib.bonsai_lowbit_gemm_host(P, H, H, 4, 4, 128, 2, H, H, H, P) == 1  # null host input
     assert lib.bonsai_lowbit_gemm_host(H, H, H, 4, 4, 128, 2, H, P, H, P) == 1  # null work buffer
     assert lib.bonsai_lowbit_gemm_host(H, H, H, 4, 4, 128, 2, H, 8, H, P) == 3  # misaligned work buffer
+
+
+def test_batch_argument_errors_before_any_device_work(lib):
+    Prob = bw.GemmProblem
+
+    def call(problems, mode=2, count=None):
+        arr = (Prob * max(len(problems), 1))(*problems)
+        return lib.bonsai_lowbit_gemm_batch(arr, len(problems) if count is None else count, mode, None)
+
+    ok = Prob(16, 16, 16, 16, 4, 8, 128)
+    assert call([ok], mode=0) == 1  # mode
+    assert call([ok], mode=4) == 1  # the 4-bit weights have no batch form
+    assert call([ok], count=-1) == 1
+    assert lib.bonsai_lowbit_gemm_batch(None, 2, 2, None) == 1  # no array
+    assert lib.bonsai_lowbit_gemm_batch(None, 0, 2, None) == 0  # empty batch: no-op
+    assert call([Prob(None, None, None, None, 0, 8, 128), Prob(None, None, None, None, 4, 0, 256)]) == 0  # empty
+    assert call([ok, Prob(16, 16, 16, 16, 4, 8, 100)]) == 2  # K % 128 in the second problem
+    assert call([ok, Prob(16, 16, 16, 16, -1, 8, 128)]) == 2
+    assert call([Prob(16, 16, 16, 16, 1 << 31, 8, 128)]) == 2
+    assert call([ok, Prob(16, None, 16, 16, 4, 8, 128)]) == 1  # null weights with data
+    assert call([Prob(16, 16, 16, None, 4, 8, 128)]) == 1  # null out
+    assert call([ok, Prob(16, 16, 24, 16, 4, 8, 128)]) == 3  # misaligned scales
+    assert call([Prob(None, None, None, 8, 4, 8, 0)]) == 3  # K = 0 still writes out: aligned
 
 
 def test_status_strings(lib):
