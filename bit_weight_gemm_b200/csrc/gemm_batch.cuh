@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
       const int nws = (params.layer[p].K / kGroup + WG - 1) / WG;
       for (int j = 0; j < nws; ++j, ++wc) {
         const int t = wc % TT;
-        if (!(ok = warp_wait(w_empty0 + 8 * t, ((wc / TT) & 1) ^ 1, abort_flag, limit))) break;
+        if (!(ok = warp_wait_inlined(w_empty0 + 8 * t, ((wc / TT) & 1) ^ 1, abort_flag, limit))) break;
         mbar_arrive_expect_tx_elected(w_full0 + 8 * t, T::kWStageBytes);
         tma_load_2d_elected(smem_addr(slot(t)), &params.w[p], w_full0 + 8 * t, word_stage_x<MODE>(j * WG), n0);
         if (lane == 0) *last_w = wc;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
       for (int j = 0; j < nws; ++j, ++wc) {
         const int t = wc % TT;
         const int gs = groups - j * WG < WG ? groups - j * WG : WG;  // groups in this stage
-        if (!(ok = warp_wait(a_empty0 + 8 * t, ((wc / TT) & 1) ^ 1, abort_flag, limit))) break;
+        if (!(ok = warp_wait_inlined(a_empty0 + 8 * t, ((wc / TT) & 1) ^ 1, abort_flag, limit))) break;
         const uint32_t full = a_full0 + 8 * t;
         const uint32_t dst = smem_addr(slot(t) + T::kWStageBytes);
         mbar_arrive_expect_tx_elected(full, static_cast<uint32_t>(gs * T::kActGroupBytes));
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
     float sums[BT];
     // Adds s * D of this stage's use k (its MMAs' completion) into sums.
     auto fold = [&](int k, float s) -> bool {
-      if (!warp_wait(t_free0 + 8 * turn, k & 1, abort_flag, limit)) return false;
+      if (!warp_wait_inlined(t_free0 + 8 * turn, k & 1, abort_flag, limit)) return false;
       tc_fence_after_sync();
       uint32_t v[16];
       tmem_load_16(d_cols, v);
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
               if (g < gs) sv[g >> 1] |= static_cast<uint32_t>(__ldg(srow + j * WG + g)) << (16 * (g & 1));
           }
         }
-        if (!(ok = warp_wait(w_full0 + 8 * turn, ph, abort_flag, limit))) break;
+        if (!(ok = warp_wait_inlined(w_full0 + 8 * turn, ph, abort_flag, limit))) break;
         for (int pos = 0; pos < gs; ++pos) {
           const float s_cur = scale_of(sv, pos);
           if (pend && !(ok = fold(use - 1, s_pend))) break;
@@ -337,8 +337,8 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
           if (quad == ((turn + use) & 3)) {
             // This warp issues the group's MMAs once all four quadrants have
             // converted it and the stage's activations have landed.
-            if (!(ok = warp_wait(t_ready0 + 8 * turn, use & 1, abort_flag, limit) &&
-                       warp_wait(a_full0 + 8 * turn, ph, abort_flag, limit)))
+            if (!(ok = warp_wait_inlined(t_ready0 + 8 * turn, use & 1, abort_flag, limit) &&
+                       warp_wait_inlined(a_full0 + 8 * turn, ph, abort_flag, limit)))
               break;
             tc_fence_after_sync();
             constexpr uint32_t idesc = f16_instr_desc(128, BT);
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
       if (ok && pend) ok = fold(use - 1, s_pend);
       if (!ok) break;
       // The unit's partial: the previous unit's must have been read.
-      if (ul > 0 && !(ok = warp_wait(part_free, (ul - 1) & 1, abort_flag, limit))) break;
+      if (ul > 0 && !(ok = warp_wait_inlined(part_free, (ul - 1) & 1, abort_flag, limit))) break;
 #pragma unroll
       for (int m = 0; m < BT; ++m) part[(turn * BT + m) * T::kRows + row] = sums[m];
       mbar_arrive(part_full);
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
     int p = 0, ul = 0;
     for (int u = u_begin; u < u_end; ++u, ++ul) {
       p = advance(u, p);
-      if (!warp_wait(part_full, ul & 1, abort_flag, limit)) break;
+      if (!warp_wait_inlined(part_full, ul & 1, abort_flag, limit)) break;
       uint32_t h[kRowsPerThread][BT / 2];  // FP16 pairs (token 2j, 2j+1) of each row
 #pragma unroll
       for (int r = 0; r < kRowsPerThread; ++r) {

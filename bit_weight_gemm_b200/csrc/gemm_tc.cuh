@@ -258,6 +258,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
+// warp_wait with the blocking loop inlined (see wait_phase_inlined).
+__device__ __forceinline__ bool warp_wait_inlined(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint64_t limit_ns) {
+  const bool ok = wait_phase_inlined(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Reads 8 columns of this thread's lane from each of the NACC accumulators
 // (BLOCK_T columns apart) and adds the first `used` of them in a fixed order
 // (an accumulator no MMA wrote holds nothing meaningful).

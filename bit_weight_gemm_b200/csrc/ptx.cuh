@@ -115,9 +115,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// The blocking part of wait_phase, kept out of line.
-__device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                             uint64_t limit_ns) {
+// The blocking loop of a bounded wait.
+__device__ __forceinline__ bool wait_phase_loop(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -132,6 +132,12 @@ __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, vola
   }
 }
 
+// The blocking part of wait_phase, kept out of line.
+__device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             uint64_t limit_ns) {
+  return wait_phase_loop(bar, parity, abort_flag, limit_ns);
+}
+
 // Waits until the phase with the given parity of barrier `bar` completes.
 // Returns false (without waiting further) when the CTA's abort flag is up or
 // when `limit_ns` has passed; in the latter case it records the timeout.
@@ -140,6 +146,14 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
                                            uint64_t limit_ns) {
   if (mbar_test_wait(bar, parity)) return true;
   return wait_phase_slow(bar, parity, abort_flag, limit_ns);
+}
+
+// The same wait with its loop inlined, for kernels whose waits mostly block
+// (the batched small-M kernel: a call per wait measured 8% of its time).
+__device__ __forceinline__ bool wait_phase_inlined(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                   uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return wait_phase_loop(bar, parity, abort_flag, limit_ns);
 }
 
 // ------------------------------------------- programmatic dependent launch --
