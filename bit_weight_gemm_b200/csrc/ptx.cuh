@@ -346,6 +346,50 @@ __device__ __forceinline__ void mma_f16_tmem_a_elected(uint32_t d_tmem, uint32_t
       : "memory");
 }
 
+// The 8 MMAs of one 128-wide K group (K=16 each), issued by one elected
+// lane: A from TMEM columns a_tmem + 8kk, B from SW128 K slices of SLICE
+// bytes (descriptor start addresses advance by 32 bytes within a slice and by
+// SLICE bytes between the two).  The first MMA overwrites D.
+template <int SLICE>
+__device__ __forceinline__ void mma8_f16_tmem_a_elected(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                        uint32_t idesc) {
+  static_assert(SLICE % 16 == 0 && SLICE / 16 + 6 < (1 << 14), "descriptor start-address offsets");
+  asm volatile(
+      "{\n"
+      "  .reg .pred e, f, t;\n"
+      "  .reg .b64 b1, b2, b3, b4, b5, b6, b7;\n"
+      "  .reg .b32 a1, a2, a3, a4, a5, a6, a7;\n"
+      "  setp.ne.b32 f, %3, %3;\n"
+      "  setp.eq.b32 t, %3, %3;\n"
+      "  add.s64 b1, %2, 2;\n"
+      "  add.s64 b2, %2, 4;\n"
+      "  add.s64 b3, %2, 6;\n"
+      "  add.s64 b4, %2, %4;\n"
+      "  add.s64 b5, %2, %5;\n"
+      "  add.s64 b6, %2, %6;\n"
+      "  add.s64 b7, %2, %7;\n"
+      "  add.u32 a1, %1, 8;\n"
+      "  add.u32 a2, %1, 16;\n"
+      "  add.u32 a3, %1, 24;\n"
+      "  add.u32 a4, %1, 32;\n"
+      "  add.u32 a5, %1, 40;\n"
+      "  add.u32 a6, %1, 48;\n"
+      "  add.u32 a7, %1, 56;\n"
+      "  elect.sync _|e, 0xffffffff;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, f;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b4, %3, t;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b5, %3, t;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b6, %3, t;\n"
+      "  @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b7, %3, t;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "n"(SLICE / 16), "n"(SLICE / 16 + 2), "n"(SLICE / 16 + 4),
+      "n"(SLICE / 16 + 6)
+      : "memory");
+}
+
 // The elected lane (the one that issued the MMAs) commits.
 __device__ __forceinline__ void mma_commit_elected(uint32_t bar) {
   asm volatile(
