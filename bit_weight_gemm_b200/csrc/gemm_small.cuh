@@ -303,14 +303,9 @@ __global__ void __launch_bounds__(SmallTile<MODE>::kThreads, 1)
           break;
         tc_fence_after_sync();
         constexpr uint32_t idesc = f16_instr_desc(128, BT);
-        const uint64_t desc_g = sw128_kmajor_desc(smem_addr(smem + T::kActOff + i * T::kActGroupBytes));
-        const uint32_t a_cols = tmem + 64 * turn;
-        const uint32_t d_col = tmem + T::kAccCol0 + 16 * turn;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bdesc = desc_g + static_cast<uint64_t>(((kk >> 2) * T::kSliceBytes + (kk & 3) * 32) >> 4);
-          mma_f16_tmem_a_elected(d_col, a_cols + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
-        }
+        mma8_f16_tmem_a_elected<T::kSliceBytes>(
+            tmem + T::kAccCol0 + 16 * turn, tmem + 64 * turn,
+            sw128_kmajor_desc(smem_addr(smem + T::kActOff + i * T::kActGroupBytes)), idesc);
         mma_commit_elected(t_free0 + 8 * turn);
         if (lane == 0) issued_uses[turn] = k + 1;
       }
