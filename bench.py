@@ -547,11 +547,15 @@ def time_small_batch(torch, bw, args, dist, peaks, peaks_kind):
         achieved = nbytes / per_call / 1e9
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         flop = sum(2 * 16 * n * k for n, k in shapes)
+        # DRAM bytes: captured per layer on a 24-layer batch of one shape, times the layers
+        per_layer = ncu_traffic(f"batch_ternary_M16_N{shapes[0][0]}_K{shapes[0][1]}_per_layer") \
+            if len(set(shapes)) == 1 else None
         out.append({"workload": name, "M": 16, "layers": len(shapes), "value": achieved, "unit": "GB/s",
                     "us_per_call": per_call * 1e6, "us_per_layer": per_call * 1e6 / len(shapes),
                     "tflops": flop / per_call / 1e12, "api": "bonsai_lowbit_gemm_batch, one call per step",
                     "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                                 "frac": achieved / peak, "traffic": ncu_traffic(f"batch_{name}"),
+                                 "frac": achieved / peak,
+                                 "traffic": per_layer * len(shapes) if per_layer is not None else None,
                                  "algorithmic_bytes_per_call": nbytes, "peak_source": f"{peaks_kind} hbm copy"},
                     "gpu_launches": steps})
         del probs, outs, base
