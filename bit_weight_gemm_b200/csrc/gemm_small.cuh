@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(SmallTile<MODE>::kThreads, 1)
     bool ok = true;
     // Adds s * D of this stage's finished group (its use `use`) into sums.
     auto fold = [&](int use, float s) -> bool {
-      if (!warp_wait(t_free0 + 8 * turn, use & 1, abort_flag, limit)) return false;
+      if (!warp_wait_inlined(t_free0 + 8 * turn, use & 1, abort_flag, limit)) return false;
       tc_fence_after_sync();
       uint32_t v[16];
       tmem_load_16(d_cols, v);
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(SmallTile<MODE>::kThreads, 1)
       if (!ok || i >= ng) break;
       if (k > 0 && !(ok = fold(k - 1, sc[k - 1]))) break;
       const int wj = i / T::kWGroups, pos = i % T::kWGroups;
-      if (!(ok = warp_wait(w_full0 + 8 * wj, 0, abort_flag, limit))) break;
+      if (!(ok = warp_wait_inlined(w_full0 + 8 * wj, 0, abort_flag, limit))) break;
       const uint8_t* wrow = smem + T::kWOff + wj * T::kWStageBytes + row * T::kWRowBytes;
       uint32_t words[T::kWordsPerGroup];
       if constexpr (T::kB3) {
@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(SmallTile<MODE>::kThreads, 1)
       if (quad == ((turn + k) & 3)) {
         // This warp issues the group's MMAs once all four quadrants have
         // converted it and its activations have landed.
-        if (!(ok = warp_wait(t_ready0 + 8 * turn, k & 1, abort_flag, limit) &&
-                   warp_wait(a_full0 + 8 * i, 0, abort_flag, limit)))
+        if (!(ok = warp_wait_inlined(t_ready0 + 8 * turn, k & 1, abort_flag, limit) &&
+                   warp_wait_inlined(a_full0 + 8 * i, 0, abort_flag, limit)))
           break;
         tc_fence_after_sync();
         constexpr uint32_t idesc = f16_instr_desc(128, BT);
