@@ -558,6 +558,7 @@ constexpr TileCost tile_cost(int block_t) {
   return block_t <= 32    ? TileCost{0.31, 1.5, 1.0}
          : block_t == 64  ? TileCost{0.31, 2.0, 1.5}
          : block_t == 128 ? TileCost{0.50, 2.5, 2.0}
+         : block_t == 176 ? TileCost{0.59, 2.7, 2.75}  // interpolated between 128 and 192
          : block_t == 192 ? TileCost{0.62, 2.75, 3.0}
                           : TileCost{0.75, 3.0, 4.0};
 }
@@ -585,6 +586,10 @@ void consider(int M, int N, int K, Plan* best) {
     const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T>(ks);
     if (per_wave <= 0) continue;
     const int waves = (tiles + per_wave - 1) / per_wave;
+    // 176-token tiles only where they fit one wave (1024 tokens on the N=3072
+    // layers); with more tiles the persistent 192- or 256-token forms win
+    // (measured at 2048 tokens, N=3072, K=9216: 1068 TFLOP/s against ~1300).
+    if (BLOCK_T == 176 && waves > 1) continue;
     bool persistent = false;
     if constexpr (BLOCK_T >= 192) persistent = ks == 1 && use_persistent<MODE, BLOCK_T>(M, N, K);
     const double per_wave_cost = ((groups + ks - 1) / ks) * c.group + (persistent ? kPersistentBoundary : c.wave) +
@@ -602,10 +607,11 @@ void consider(int M, int N, int K, Plan* best) {
 }
 
 // Tokens per tile: the smallest MMA N that covers M up to 128; above that
-// 128-, 192- or 256-token tiles, whichever the cost model prefers (256
-// amortises each converted weight over the most tokens; 192 and 128 waste
-// fewer rows and fill more SMs at mid M: M=1024 with N=3072 makes 96
-// 256-token tiles for 148 SMs but 144 192-token ones).
+// 128-, 176-, 192- or 256-token tiles, whichever the cost model prefers (256
+// amortises each converted weight over the most tokens; the narrower ones
+// waste fewer rows and fill more SMs at mid M: M=1024 with N=3072 makes 96
+// 256-token tiles for 148 SMs but 144 of 192 or 176 tokens, and 176-token
+// tiles leave 32 empty token rows where 192-token ones leave 128).
 template <int MODE>
 Plan plan_gemm(int M, int N, int K) {
   Plan best;
@@ -627,6 +633,7 @@ Plan plan_gemm(int M, int N, int K) {
     consider<MODE, 128>(M, N, K, &best);
   } else {
     consider<MODE, 128>(M, N, K, &best);
+    consider<MODE, 176>(M, N, K, &best);
     consider<MODE, 192>(M, N, K, &best);
     consider<MODE, 256>(M, N, K, &best);
   }
@@ -648,6 +655,7 @@ int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales,
     case 32: return launch_gemm<MODE, 32>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 64: return launch_gemm<MODE, 64>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 128: return launch_gemm<MODE, 128>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+    case 176: return launch_gemm<MODE, 176>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 192: return launch_gemm<MODE, 192>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 256: return launch_gemm<MODE, 256>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     default: return BONSAI_ERR_CUDA;  // no plan: the occupancy queries failed

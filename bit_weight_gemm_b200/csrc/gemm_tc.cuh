@@ -82,7 +82,7 @@ struct GemmTile {
   // Activation stages: as many as fit next to the word ring and the scales,
   // so that narrow tiles keep a split-K CTA's whole K range in flight.
   static constexpr int kActStages =
-      BLOCK_T >= 192 ? 3 : (BLOCK_T >= 128 ? 4 : (96 * 1024) / kActStageBytes);
+      BLOCK_T > 128 ? 3 : (BLOCK_T == 128 ? 4 : (96 * 1024) / kActStageBytes);
   // A word stage is 128 bytes of every row: 4 ternary or 8 binary groups,
   // one TMA box with 128-byte swizzling.
   // Base-3: one 112-byte block (4 groups) of every row per stage, without
@@ -95,7 +95,7 @@ struct GemmTile {
   static constexpr int kGroupAlign = kB3 ? kB3BlockGroups : 1;
   // Small token tiles are bandwidth-bound: enough word stages to keep every
   // load of a split-K CTA in flight at once.
-  static constexpr int kWStages = BLOCK_T >= 192 ? 2 : 4;
+  static constexpr int kWStages = BLOCK_T > 128 ? 2 : 4;
   // The tile's scales, staged once per CTA when 128 x groups x 2 bytes fit.
   // (4-bit group-affine weights keep scale and zero pairs in registers.)
   static constexpr int kScaleBytes = (BLOCK_T >= 256 || kHqq) ? 0 : 32768;

@@ -198,8 +198,8 @@ def _sms():
 def test_plans_cover_every_form():
     big = bw.gemm_plan(4608, 9216, 3072, "ternary")  # persistent: one CTA per SM walks 1296 tiles
     assert big == {"block_t": 256, "ksplit": 1, "ctas": _sms(), "tiles": 72 * 18}
-    one_wave = bw.gemm_plan(1024, 3072, 3072, "binary")  # 144 192-token tiles: one CTA each, one wave
-    assert one_wave["block_t"] == 192 and one_wave["tiles"] == 24 * 6
+    one_wave = bw.gemm_plan(1024, 3072, 3072, "binary")  # 144 176-token tiles: one CTA each, one wave
+    assert one_wave["block_t"] == 176 and one_wave["tiles"] == 24 * 6
     assert one_wave["ctas"] == one_wave["tiles"] * one_wave["ksplit"]
     for M, N, K in [(16, 3072, 9216), (16, 256, 4096), (40, 384, 2048)]:
         p = bw.gemm_plan(M, N, K, "ternary")
@@ -243,23 +243,26 @@ LARGE_M_SHAPES = [
 ]
 
 
-# 192-token tiles, where 256-token ones would leave SMs idle: one wave of
-# one-tile CTAs (M=1024 / 1000 with N=3072 / 3000: 144 tiles) and the
-# persistent kernel (M=2048 with N=3072: 264 tiles); ragged M and N.
-TILE192_SHAPES = [
-    ("binary", 1024, 3072, 3072, False),
-    ("ternary", 1000, 3000, 1152, False),
-    ("ternary_b3", 1000, 3000, 1152, False),
-    ("ternary", 2048, 3072, 2048, True),
-    ("ternary_b3", 2000, 3050, 2048, True),
-    ("binary", 2048, 3072, 2048, True),
+# Mid-M token tiles, where 256-token ones would leave SMs idle: one wave of
+# one-tile CTAs of 176 tokens (M=1024 / 1000 with N=3072 / 3000: 144 tiles)
+# and the persistent kernel with 192-token tiles (M=2048 with N=3072: 264
+# tiles); ragged M and N, in every format (the 4-bit weights at 1000 x 3000
+# in test_hqq4_gemm_full).
+MID_M_TILE_SHAPES = [
+    ("binary", 1024, 3072, 3072, 176, False),
+    ("ternary", 1000, 3000, 1152, 176, False),
+    ("ternary_b3", 1000, 3000, 1152, 176, False),
+    ("ternary", 1024, 3072, 12288, 176, False),
+    ("ternary", 2048, 3072, 2048, 192, True),
+    ("ternary_b3", 2000, 3050, 2048, 192, True),
+    ("binary", 2048, 3072, 2048, 192, True),
 ]
 
 
-@pytest.mark.parametrize("mode,M,N,K,persistent", TILE192_SHAPES)
-def test_gemm_192_token_tiles(oracle_mod, mode, M, N, K, persistent):
+@pytest.mark.parametrize("mode,M,N,K,block_t,persistent", MID_M_TILE_SHAPES)
+def test_gemm_mid_m_token_tiles(oracle_mod, mode, M, N, K, block_t, persistent):
     plan = bw.gemm_plan(M, N, K, mode)
-    assert plan["block_t"] == 192 and plan["ksplit"] == 1, plan
+    assert plan["block_t"] == block_t and plan["ksplit"] == 1, plan
     assert (plan["ctas"] < plan["tiles"]) == persistent, plan
     got, ref, absacc = _gemm_case(oracle_mod, mode, M, N, K, seed=M + 5 * N + 3 * K)
     assert_gemm_close(oracle_mod, got, ref, absacc, f"{mode} {M}x{N}x{K}")
