@@ -6,8 +6,9 @@ call, every problem compared with the CPU oracle through the C ABI.
   larger-M, K = 0 and empty problems among them;
 - more problems than one launch takes (so the batch is cut in two);
 - scales with negatives, signed zeros, subnormals and large magnitudes;
-- the 80 linears of one denoise step at 16 tokens in one call, and 80
-  MLP-down layers (3072x9216) at 16 tokens, as the benchmark times them;
+- the 80 linears of one denoise step at 16 tokens in one call, in every
+  storage format, and 80 MLP-down layers (3072x9216) at 16 tokens, as the
+  benchmark times them;
 - a batch captured in a CUDA graph and replayed.
 
 Bar as everywhere: |gpu - oracle| <= 1e-3 * sum_k |a_k w_k| + one FP16 ulp
@@ -160,7 +161,7 @@ def _positions(M, N, count, seed):
     return np.array(ms, np.int64), np.array(ns, np.int64)
 
 
-def _layers(oracle_mod, shapes, M, seed, distinct_codes=4):
+def _layers(oracle_mod, shapes, M, seed, distinct_codes=4, mode="ternary"):
     """Problems of the given (N, K) at M tokens: own activations and scales
     each, codes shared among every distinct_codes-th layer of a shape."""
     codes = {}
@@ -169,8 +170,8 @@ def _layers(oracle_mod, shapes, M, seed, distinct_codes=4):
     for j, (n, k) in enumerate(shapes):
         key = (n, k, j % distinct_codes)
         if key not in codes:
-            d = workloads.make(mode="ternary", M=1, N=n, K=k, seed=seed + 1 + len(codes))
-            codes[key] = (bw.pack(dev(d["codes"]), "ternary"), oracle_mod.pack(d["codes"], "ternary"))
+            d = workloads.make(mode=mode, M=1, N=n, K=k, seed=seed + 1 + len(codes))
+            codes[key] = (bw.pack(dev(d["codes"]), mode), oracle_mod.pack(d["codes"], mode))
         a = workloads.activations(rng, M, k)
         s = workloads.scales(rng, n, k)
         probs.append({"a": a, "s_np": s, "A": dev(a.view(np.int16), torch.float16), "packed": codes[key][0],
@@ -179,32 +180,36 @@ def _layers(oracle_mod, shapes, M, seed, distinct_codes=4):
     return probs
 
 
-def _check_sampled(oracle_mod, probs, outs, M, label, full=()):
+def _check_sampled(oracle_mod, probs, outs, M, label, full=(), mode="ternary"):
     for j, (p, out) in enumerate(zip(probs, outs)):
         got = to_u16(out)
         assert not np.isnan(got.view(np.float16)).any(), f"{label} {j}: an output was not written"
         if j in full:
-            ref, _, absacc = oracle_mod.gemm(p["a"], p["ref_packed"], p["s_np"], p["K"], "ternary")
+            ref, _, absacc = oracle_mod.gemm(p["a"], p["ref_packed"], p["s_np"], p["K"], mode)
             check(oracle_mod, got, ref, absacc, f"{label} {j} (every output)")
             continue
         ms, ns = _positions(M, p["N"], 300, j)
-        ref, _, absacc = oracle_mod.gemm_entries(p["a"], p["ref_packed"], p["s_np"], p["K"], "ternary", ms, ns)
+        ref, _, absacc = oracle_mod.gemm_entries(p["a"], p["ref_packed"], p["s_np"], p["K"], mode, ms, ns)
         check(oracle_mod, got[ms, ns], ref, absacc, f"{label} {j}")
 
 
-def test_denoise_step_linears_at_16_tokens(oracle_mod):
+@pytest.mark.parametrize("mode", MODES)
+def test_denoise_step_linears_at_16_tokens(oracle_mod, mode):
     """The 80 linears of one denoise step (Q|K|V stacked) at 16 tokens, in
-    one call: one persistent launch over 2592 weight tiles."""
+    one call: one persistent launch over 2592 weight tiles, in every storage
+    format (binary: 8 groups per word stage, two-turn slots of 48 KB;
+    base-3: 112-byte blocks)."""
     layers = workloads.mmdit_stack_layers()
-    probs = _layers(oracle_mod, [(n, k) for _, n, k in layers], 16, 7400)
+    probs = _layers(oracle_mod, [(n, k) for _, n, k in layers], 16, 7400 + MODES.index(mode), mode=mode)
     outs = [torch.full((16, p["N"]), float("nan"), dtype=torch.float16, device="cuda") for p in probs]
-    bw.lowbit_gemm_batch([(p["A"], p["packed"], p["s"]) for p in probs], "ternary", outs=outs)
+    bw.lowbit_gemm_batch([(p["A"], p["packed"], p["s"]) for p in probs], mode, outs=outs)
     torch.cuda.synchronize()
     # every output of one layer of each shape, sampled positions of the rest
     first = {}
     for j, p in enumerate(probs):
         first.setdefault((p["N"], p["K"]), j)
-    _check_sampled(oracle_mod, probs, outs, 16, "denoise-step linear", full=set(first.values()))
+    _check_sampled(oracle_mod, probs, outs, 16, f"{mode} denoise-step linear", full=set(first.values()),
+                   mode=mode)
 
 
 def test_mlp_down_batch_at_16_tokens(oracle_mod):
