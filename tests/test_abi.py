@@ -129,6 +129,19 @@ def test_batch_argument_errors_before_any_device_work(lib):
     assert call([Prob(None, None, None, 8, 4, 8, 0)]) == 3  # K = 0 still writes out: aligned
 
 
+def test_c_program_uses_the_abi(lib, tmp_path):
+    """A C99 program built against include/bonsai.h and linked with
+    libbonsai.so gets the documented sizes, status strings and argument
+    errors (no device work, so it runs without a GPU)."""
+    exe = tmp_path / "abi_check"
+    libdir = os.path.dirname(bw.library_path())
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi_check.c"), "-L", libdir, "-lbonsai",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", res.stderr
+
+
 def test_status_strings(lib):
     for s in range(8):
         assert bw.status_string(s) != "unknown status"
