@@ -496,23 +496,29 @@ def time_small_batch(torch, bw, args, dist, peaks, peaks_kind):
     launch), each layer with its own buffers (633-752 MB in all, 5-6x L2, so
     every weight byte comes from HBM).  Three batches: 80 MLP-down layers
     (3072x9216), 80 fused-QKV layers (9216x3072), and the 80 linears of one
-    denoise step.  GB/s of algorithmic bytes (packed weights, scales,
+    denoise step; then the two repeated-layer batches with binary weights and
+    MLP-down with base-3 ternary weights.  GB/s of algorithmic bytes (packed weights, scales,
     activations, outputs of all layers) per call; the call is replayed from a
     CUDA graph and timed with CUDA events on the replay stream."""
     out = []
     step_layers = [(n, k) for _, n, k in workloads.mmdit_stack_layers()]
-    cases = [("ternary MLP-down M=16 x 80 layers", [(SMALL[0].N, SMALL[0].K)] * BATCH_LAYERS, SMALL[0].seed),
-             ("ternary fused QKV M=16 x 80 layers", [(SMALL[1].N, SMALL[1].K)] * BATCH_LAYERS, SMALL[1].seed),
-             ("ternary denoise-step linears M=16 (80 layers)", step_layers, 3000)]
-    for name, shapes, seed in cases:
+    down = [(SMALL[0].N, SMALL[0].K)] * BATCH_LAYERS
+    qkv = [(SMALL[1].N, SMALL[1].K)] * BATCH_LAYERS
+    cases = [("ternary MLP-down M=16 x 80 layers", "ternary", down, SMALL[0].seed),
+             ("ternary fused QKV M=16 x 80 layers", "ternary", qkv, SMALL[1].seed),
+             ("ternary denoise-step linears M=16 (80 layers)", "ternary", step_layers, 3000),
+             ("binary MLP-down M=16 x 80 layers", "binary", down, SMALL[0].seed),
+             ("binary fused QKV M=16 x 80 layers", "binary", qkv, SMALL[1].seed),
+             ("base-3 ternary MLP-down M=16 x 80 layers", "ternary_b3", down, SMALL[0].seed)]
+    for name, mode, shapes, seed in cases:
         base = {}
         probs, nbytes = [], 0
         for j, (n, k) in enumerate(shapes):
-            p = workloads.Problem(name, "ternary", 16, n, k, seed + j)
+            p = workloads.Problem(name, mode, 16, n, k, seed + j)
             if (n, k) not in base:
                 d = workloads.make(p)
                 base[(n, k)] = (torch.from_numpy(d["A"].view(np.int16)).view(torch.float16).cuda(),
-                                bw.pack(torch.from_numpy(d["codes"]).cuda(), "ternary"),
+                                bw.pack(torch.from_numpy(d["codes"]).cuda(), mode),
                                 torch.from_numpy(d["scales"].view(np.int16)).view(torch.float16).cuda())
             A, packed, sc = (t.clone() for t in base[(n, k)])  # own buffers: every layer reads its own bytes
             probs.append((A, packed, sc))
@@ -521,7 +527,7 @@ def time_small_batch(torch, bw, args, dist, peaks, peaks_kind):
         torch.cuda.synchronize()
 
         def call():
-            bw.lowbit_gemm_batch(probs, "ternary", outs=outs)
+            bw.lowbit_gemm_batch(probs, mode, outs=outs)
 
         for _ in range(max(args.warmup, 3)):
             call()
@@ -548,9 +554,9 @@ def time_small_batch(torch, bw, args, dist, peaks, peaks_kind):
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         flop = sum(2 * 16 * n * k for n, k in shapes)
         # DRAM bytes: captured per layer on a 24-layer batch of one shape, times the layers
-        per_layer = ncu_traffic(f"batch_ternary_M16_N{shapes[0][0]}_K{shapes[0][1]}_per_layer") \
+        per_layer = ncu_traffic(f"batch_{mode}_M16_N{shapes[0][0]}_K{shapes[0][1]}_per_layer") \
             if len(set(shapes)) == 1 else None
-        out.append({"workload": name, "M": 16, "layers": len(shapes), "value": achieved, "unit": "GB/s",
+        out.append({"workload": name, "mode": mode, "M": 16, "layers": len(shapes), "value": achieved, "unit": "GB/s",
                     "us_per_call": per_call * 1e6, "us_per_layer": per_call * 1e6 / len(shapes),
                     "tflops": flop / per_call / 1e12, "api": "bonsai_lowbit_gemm_batch, one call per step",
                     "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

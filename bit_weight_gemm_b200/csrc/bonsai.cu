@@ -500,7 +500,12 @@ int launch_gemm_batch(const bonsai_gemm_problem* const* probs, int count, cudaSt
     if (!make_map(&params.act[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q.A, K, M, 64, T::kBlockT,
                   CU_TENSOR_MAP_SWIZZLE_128B))
       return BONSAI_ERR_CUDA;
-    if (!make_weight_map(&params.w[i], q.packed, N, K, MODE)) return BONSAI_ERR_CUDA;
+    // Binary word stages are 64-byte rows (four groups), the others as in the other kernels.
+    if (MODE == BONSAI_BINARY ? !make_map(&params.w[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, q.packed,
+                                          static_cast<uint64_t>(row_words(K, MODE)), N, T::kWRowBytes / 4, 128,
+                                          CU_TENSOR_MAP_SWIZZLE_64B)
+                              : !make_weight_map(&params.w[i], q.packed, N, K, MODE))
+      return BONSAI_ERR_CUDA;
     params.layer[i] = BatchLayer{q.scales, q.out, M, N, K, units};
     const int tiles = (N + T::kRows - 1) / T::kRows;
     units += tiles;

@@ -14,9 +14,9 @@
 // tensor memory takes a whole SM, so consecutive launches do not overlap).
 // Here one CTA per SM walks a list of units, a unit being one layer's
 // 128-row tile over the whole of K, and the rings run on across units and
-// layers.  The CTA's word stages (128 bytes of each of the 128 rows: 4 INT2,
-// 8 binary or one 112-byte block of 4 base-3 groups) are dealt out in turn:
-// stage wc goes to slot and turn wc mod T (T = 5, or 4 for binary weights),
+// layers.  The CTA's word stages (four groups of each of the 128 rows: 128
+// bytes INT2, 64 binary, one 112-byte block base-3) are dealt out in turn:
+// stage wc goes to slot and turn wc mod T (T = 5),
 // so every barrier of a slot serves the same warps, phase after phase.
 //
 //   warp 0     TMA of each stage's packed words into its slot, issued before
@@ -71,17 +71,18 @@ struct BatchTile {
   static constexpr int kRows = 128;   // weight rows (MMA M)
   static constexpr bool kB3 = MODE == BONSAI_TERNARY_B3;
   static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : 8);  // held per group
-  static constexpr int kWGroups = kB3 ? kB3BlockGroups : 32 / kWordsPerGroup;        // groups per word stage
-  static constexpr int kWRowBytes = kB3 ? kB3BlockBytes : 128;
+  static constexpr int kWGroups = 4;                                                  // groups per word stage
+  static constexpr int kWRowBytes = kB3 ? kB3BlockBytes : 16 * kWordsPerGroup;  // binary: 64 (64-byte swizzle)
   static constexpr int kWStageBytes = kRows * kWRowBytes;
   static constexpr int kSliceBytes = kBlockT * 128;       // 16 rows x 64 FP16, one SW128 K slice
   static constexpr int kActGroupBytes = 2 * kSliceBytes;  // one group's activations
   // A turn's slot: one word stage and the activations of its groups.
   static constexpr int kSlotBytes = kWStageBytes + kWGroups * kActGroupBytes;
   // Turns (converter warps per lane quadrant = slots = TMEM stages), as many
-  // as shared memory holds: 5 (32 KB slots; 30 KB base-3) or 4 (binary: 8
-  // groups per stage, 48 KB slots).
-  static constexpr int kTurns = MODE == BONSAI_BINARY ? 4 : 5;
+  // as shared memory holds: 5 (32 KB slots; 30 KB base-3, 24 KB binary).
+  // Warps are what hide the hand-over latencies: binary weights in 8-group
+  // stages, with room for 4 turns only, ran 43% longer per layer than INT2.
+  static constexpr int kTurns = 5;
   static constexpr int kConvWarp0 = 2;
   static constexpr int kConvWarps = 4 * kTurns;
   static constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps;
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
     bool ok = true;
     // The stage's scales of this row, FP16 pairs: groups 2i, 2i+1 in sv[i].
     constexpr int kSv = WG / 2;
+    static_assert(kSv == 2, "a stage's scales are one 8-byte load");
     auto scale_of = [&](const uint32_t* sv, int pos) -> float {
       uint32_t h = sv[0];
 #pragma unroll
@@ -282,17 +284,9 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
         for (int i = 0; i < kSv; ++i) sv[i] = 0u;
         if (row_in) {
           if (vec_scales) {
-            if constexpr (kSv == 4) {
-              const uint4 q = __ldg(reinterpret_cast<const uint4*>(srow + j * WG));
-              sv[0] = q.x;
-              sv[1] = q.y;
-              sv[2] = q.z;
-              sv[3] = q.w;
-            } else {
-              const uint2 q = __ldg(reinterpret_cast<const uint2*>(srow + j * WG));
-              sv[0] = q.x;
-              sv[1] = q.y;
-            }
+            const uint2 q = __ldg(reinterpret_cast<const uint2*>(srow + j * WG));
+            sv[0] = q.x;
+            sv[1] = q.y;
           } else {
 #pragma unroll
             for (int g = 0; g < WG; ++g)
@@ -306,8 +300,8 @@ __global__ void __launch_bounds__(BatchTile<MODE>::kThreads, 1)
           uint32_t words[T::kWordsPerGroup];
           if constexpr (T::kB3) {
             b3_group_words(reinterpret_cast<const uint32_t*>(wslot), pos, words);
-          } else if (MODE == BONSAI_BINARY) {
-            const uint4 q = *reinterpret_cast<const uint4*>(wslot + 16 * (pos ^ (row & 7)));
+          } else if (MODE == BONSAI_BINARY) {  // 64-byte rows, 64-byte swizzle
+            const uint4 q = *reinterpret_cast<const uint4*>(wslot + 16 * (pos ^ ((row >> 1) & 3)));
             words[0] = q.x;
             words[1] = q.y;
             words[2] = q.z;

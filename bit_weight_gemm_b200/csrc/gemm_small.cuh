@@ -104,13 +104,15 @@ struct SmallArgs {
 template <int MODE>
 __device__ __forceinline__ void convert_group_unscaled(const uint32_t* words, uint32_t taddr) {
   if (MODE == BONSAI_BINARY) {
+    // One logic instruction per pair besides the shift: the sign bits under
+    // the sign mask, or'ed with 1.0's exponent (both masks kept in registers).
+    const uint32_t sign = 0x80008000u, one = 0x3C003C00u;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t v[16];
+    for (int c = 0; c < 8; ++c) {
+      uint32_t v[8];
 #pragma unroll
-      for (int p = 0; p < 16; ++p) v[p] = ((words[j] << p) & 0x80008000u) | 0x3C003C00u;
-      tmem_store_8(taddr + j * 16, v);
-      tmem_store_8(taddr + j * 16 + 8, v + 8);
+      for (int p = 0; p < 8; ++p) v[p] = and_or(words[c >> 1] << (8 * (c & 1) + p), sign, one);
+      tmem_store_8(taddr + c * 8, v);
     }
   } else if (MODE == BONSAI_TERNARY_B3) {
     uint32_t y[13];
