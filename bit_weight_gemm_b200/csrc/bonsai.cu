@@ -792,12 +792,17 @@ int bonsai_pack(const int8_t* codes, int64_t N, int64_t K, int mode, void* packe
   if (cudaMemcpyToSymbolAsync(g_pack_bad_code, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return BONSAI_ERR_CUDA;
   if (mode == BONSAI_TERNARY_B3) {
-    const int64_t blocks = N * (row_words(K, mode) / (kB3BlockBytes / 4));
-    pack_b3_kernel<<<grid_for(blocks, 256), 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), N, K);
+    const int64_t slots = N * (row_words(K, mode) / (kB3BlockBytes / 4)) * kB3BlockGroups;
+    if ((reinterpret_cast<uintptr_t>(codes) & 31u) == 0)
+      pack_b3_kernel<true><<<grid_for(slots, 256), 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), N, K);
+    else
+      pack_b3_kernel<false><<<grid_for(slots, 256), 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), N, K);
   } else {
     const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
-    const int grid = grid_for(words / 8, 256);  // two 4-word steps per thread
-    if (mode == BONSAI_BINARY)
+    const int grid = grid_for(words / (mode == BONSAI_BINARY ? 4 : 8), 256);  // 4-word steps: one binary, two ternary
+    if (mode == BONSAI_BINARY && (reinterpret_cast<uintptr_t>(codes) & 31u) == 0)
+      pack_kernel<BONSAI_BINARY, true><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
+    else if (mode == BONSAI_BINARY)
       pack_kernel<BONSAI_BINARY><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
     else
       pack_kernel<BONSAI_TERNARY_INT2><<<grid, 256, 0, st>>>(codes, static_cast<uint32_t*>(packed), words);
@@ -827,10 +832,16 @@ int bonsai_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_
   }
   const int64_t words = N * K / (mode == BONSAI_BINARY ? 32 : 16);
   const int grid = grid_for(words, 256);
-  if (mode == BONSAI_BINARY)
-    dequant_kernel<BONSAI_BINARY><<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(packed), scales, w, N, K);
+  const auto* pk = static_cast<const uint32_t*>(packed);
+  const bool wide = (reinterpret_cast<uintptr_t>(w) & 31u) == 0;  // 32-byte stores
+  if (mode == BONSAI_BINARY && wide)
+    dequant_kernel<BONSAI_BINARY, true><<<grid, 256, 0, st>>>(pk, scales, w, N, K);
+  else if (mode == BONSAI_BINARY)
+    dequant_kernel<BONSAI_BINARY, false><<<grid, 256, 0, st>>>(pk, scales, w, N, K);
+  else if (wide)
+    dequant_kernel<BONSAI_TERNARY_INT2, true><<<grid, 256, 0, st>>>(pk, scales, w, N, K);
   else
-    dequant_kernel<BONSAI_TERNARY_INT2><<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(packed), scales, w, N, K);
+    dequant_kernel<BONSAI_TERNARY_INT2, false><<<grid, 256, 0, st>>>(pk, scales, w, N, K);
   return launch_status();
 }
 

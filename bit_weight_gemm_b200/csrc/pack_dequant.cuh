@@ -72,34 +72,43 @@ __device__ __forceinline__ uint32_t pack_binary_word(uint4 lo, uint4 hi, uint32_
   return w;
 }
 
-// Each thread packs 4 consecutive words per step (one 16-byte store), two
-// steps' loads in flight.  total_words is a multiple of 4 because K is a
-// multiple of 128.
-template <int MODE>
+// Each thread packs 4 consecutive words per step (one 16-byte store), with
+// eight 16-byte loads in flight: two steps for ternary codes (4 loads a
+// step), one for binary (8; as four 32-byte loads when WIDE, the codes then
+// 32-byte aligned).  total_words is a multiple of 4 because K is a multiple
+// of 128.
+template <int MODE, bool WIDE = false>
 __global__ void __launch_bounds__(256) pack_kernel(const int8_t* __restrict__ codes, uint32_t* __restrict__ packed,
                                                    int64_t total_words) {
   constexpr int kPerWord = MODE == BONSAI_BINARY ? 32 : 16;
   constexpr int kLoads = kPerWord / 4;  // 16-byte loads per 4 words
+  constexpr int kSteps = 8 / kLoads;
   const int64_t quads = total_words / 4;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   uint32_t bad = 0;
-  for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < quads; q += 2 * stride) {
-    const bool two = q + stride < quads;
-    uint4 v[2][kLoads];
-    const uint4* src = reinterpret_cast<const uint4*>(codes + q * 4 * kPerWord);
-    const uint4* src2 = reinterpret_cast<const uint4*>(codes + (two ? q + stride : q) * 4 * kPerWord);
+  for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < quads; q += kSteps * stride) {
+    uint4 v[kSteps][kLoads];
 #pragma unroll
-    for (int i = 0; i < kLoads; ++i) v[0][i] = __ldg(src + i);
+    for (int h = 0; h < kSteps; ++h) {
+      const int64_t qh = q + h * stride < quads ? q + h * stride : q;
+      const uint4* src = reinterpret_cast<const uint4*>(codes + qh * 4 * kPerWord);
+      if constexpr (WIDE) {
 #pragma unroll
-    for (int i = 0; i < kLoads; ++i) v[1][i] = __ldg(src2 + i);
+        for (int i = 0; i < kLoads; i += 2) ldg_32b(src + i, v[h][i], v[h][i + 1]);
+      } else {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+        for (int i = 0; i < kLoads; ++i) v[h][i] = __ldg(src + i);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kSteps; ++h) {
       uint32_t w[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         w[i] = MODE == BONSAI_BINARY ? pack_binary_word(v[h][2 * i], v[h][2 * i + 1], bad)
                                      : pack_ternary_word(v[h][i], bad);
-      if (h == 0 || two) reinterpret_cast<uint4*>(packed)[h == 0 ? q : q + stride] = make_uint4(w[0], w[1], w[2], w[3]);
+      if (h == 0 || q + h * stride < quads)
+        reinterpret_cast<uint4*>(packed)[q + h * stride] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
   if (!__all_sync(0xffffffffu, bad == 0) && lane_id() == 0) atomicOr(&g_pack_bad_code, 1u);
@@ -109,7 +118,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const int8_t* __restrict__ co
 // or 32 (binary) FP16 weights, 32 or 64 contiguous bytes.  The code becomes an exact FP16 t (ternary: the shifted field is 2t,
 // halved exactly; binary: the sign bit over 1.0) and one IEEE FP16 multiply
 // by the scale gives t * s with the product's sign-of-zero and NaN rules.
-template <int MODE>
+// WIDE: dst is 32-byte aligned and written 32 bytes a store.
+template <int MODE, bool WIDE>
 __device__ __forceinline__ void dequant_word(uint32_t word, uint32_t s2, uint16_t* dst) {
   constexpr int kPerWord = MODE == BONSAI_BINARY ? 32 : 16;
   uint32_t v[kPerWord / 2];
@@ -127,11 +137,18 @@ __device__ __forceinline__ void dequant_word(uint32_t word, uint32_t s2, uint16_
     }
   }
   uint4* out = reinterpret_cast<uint4*>(dst);
+  if constexpr (WIDE) {
 #pragma unroll
-  for (int i = 0; i < kPerWord / 8; ++i) out[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    for (int i = 0; i < kPerWord / 8; i += 2)
+      stg_32b(out + i, make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]),
+              make_uint4(v[4 * i + 4], v[4 * i + 5], v[4 * i + 6], v[4 * i + 7]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPerWord / 8; ++i) out[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
 }
 
-template <int MODE>
+template <int MODE, bool WIDE>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict__ packed,
                                                       const uint16_t* __restrict__ scales, uint16_t* __restrict__ w,
                                                       int64_t N, int64_t K) {
@@ -143,7 +160,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
        idx += (int64_t)gridDim.x * blockDim.x) {
     const int64_t n = idx / words_per_row, j = idx - n * words_per_row;
     const uint32_t s = __ldg(scales + n * groups + (j * kPerWord) / kGroup);
-    dequant_word<MODE>(__ldg(packed + idx), s | (s << 16), w + n * K + j * kPerWord);
+    dequant_word<MODE, WIDE>(__ldg(packed + idx), s | (s << 16), w + n * K + j * kPerWord);
   }
 }
 
@@ -263,53 +280,87 @@ __device__ __forceinline__ void b3_group_words(const uint32_t* block, int r, uin
   for (int k = 0; k < 7; ++k) w[k] = odd ? __funnelshift_r(raw[k], raw[k + 1], 16) : raw[k];
 }
 
-// Packs the codes of one row's block b (groups 4b .. 4b+3 that exist) into
-// 112 bytes.  One thread per block; codes are read as 16-byte loads.
+// Packs the codes of group slot r of one row's block b into bytes
+// 26r .. 26r+25 of the block's 112 (zeros for a slot past the row's groups;
+// bytes 104..111 are zero).  One thread per slot, so consecutive threads read
+// consecutive 128-byte groups with 16-byte loads.  A warp's 32 slots are 8
+// whole blocks (896 contiguous bytes): the threads leave their 26 bytes in a
+// shared-memory copy of them, and the warp writes it out in 16-byte stores.
+// WIDE: the codes are 32-byte aligned and read 32 bytes a load.
+template <bool WIDE>
 __global__ void __launch_bounds__(256) pack_b3_kernel(const int8_t* __restrict__ codes, uint32_t* __restrict__ packed,
                                                       int64_t N, int64_t K) {
+  constexpr int kWarpBlocks = 32 / kB3BlockGroups;
+  constexpr int kWarpBytes = kWarpBlocks * kB3BlockBytes;
+  __shared__ alignas(16) uint8_t stage_all[8][kWarpBytes];
   const int64_t groups = K / kGroup;
   const int64_t blocks_per_row = (groups + kB3BlockGroups - 1) / kB3BlockGroups;
-  const int64_t total = N * blocks_per_row;
+  const int64_t total = N * blocks_per_row * kB3BlockGroups;  // slots, a multiple of 32 / kWarpBlocks
+  const int lane = threadIdx.x & 31;
+  uint8_t* stage = stage_all[threadIdx.x >> 5];
   bool ok = true;
-  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t n = idx / blocks_per_row, b = idx - n * blocks_per_row;
-    uint32_t out[kB3BlockBytes / 4] = {};
-#pragma unroll
-    for (int r = 0; r < kB3BlockGroups; ++r) {
-      const int64_t g = b * kB3BlockGroups + r;
-      if (g >= groups) break;
+  // Warp-uniform loop over runs of 32 slots.
+  for (int64_t base = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) - lane; base < total;
+       base += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t idx = base + lane;
+    const int r = lane % kB3BlockGroups;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(stage + (lane / kB3BlockGroups) * kB3BlockBytes + kB3GroupBytes * r);
+    const int64_t blk = idx / kB3BlockGroups;  // n * blocks_per_row + b
+    const int64_t n = blk / blocks_per_row;
+    const int64_t g = (blk - n * blocks_per_row) * kB3BlockGroups + r;
+    if (idx < total && g < groups) {
       const uint4* src = reinterpret_cast<const uint4*>(codes + n * K + g * kGroup);
+      uint4 q4[8];
+      if constexpr (WIDE) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) ldg_32b(src + i, q4[i], q4[i + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q4[i] = __ldg(src + i);
+      }
       uint32_t c[32];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint4 v = __ldg(src + i);
-        c[4 * i] = v.x;
-        c[4 * i + 1] = v.y;
-        c[4 * i + 2] = v.z;
-        c[4 * i + 3] = v.w;
+        c[4 * i] = q4[i].x;
+        c[4 * i + 1] = q4[i].y;
+        c[4 * i + 2] = q4[i].z;
+        c[4 * i + 3] = q4[i].w;
       }
 #pragma unroll
-      for (int j = 0; j < kB3GroupBytes; ++j) {
-        uint32_t v = 0;
+      for (int h = 0; h < kB3GroupBytes / 2; ++h) {
+        uint32_t pair = 0;
 #pragma unroll
-        for (int i = 0; i < 5; ++i) {
-          const int k = 26 * i + j;
-          uint32_t q = 0;  // positions past the group: digit 0
-          if (k < kGroup) {
-            q = ((c[k >> 2] >> (8 * (k & 3))) + 1u) & 0xFFu;  // t + 1 for t in {-1, 0, +1}
-            ok &= q <= 2u;
+        for (int e = 0; e < 2; ++e) {
+          const int j = 2 * h + e;  // byte j holds codes j, 26 + j, 52 + j, 78 + j, 104 + j
+          uint32_t v = 0;
+#pragma unroll
+          for (int i = 0; i < 5; ++i) {
+            const int k = 26 * i + j;
+            uint32_t q = 0;  // positions past the group: digit 0
+            if (k < kGroup) {
+              q = ((c[k >> 2] >> (8 * (k & 3))) + 1u) & 0xFFu;  // t + 1 for t in {-1, 0, +1}
+              ok &= q <= 2u;
+            }
+            v = 3u * v + q;
           }
-          v = 3u * v + q;
+          pair |= (((256u * v + 242u) / 243u) & 0xFFu) << (8 * e);  // ceil(256 v / 243)
         }
-        const uint32_t y = (256u * v + 242u) / 243u;  // ceil(256 v / 243)
-        const int byte = kB3GroupBytes * r + j;
-        out[byte >> 2] |= (y & 0xFFu) << (8 * (byte & 3));
+        dst[h] = static_cast<uint16_t>(pair);
       }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(packed) + idx * (kB3BlockBytes / 16);
+    } else {
 #pragma unroll
-    for (int i = 0; i < kB3BlockBytes / 16; ++i) dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+      for (int h = 0; h < kB3GroupBytes / 2; ++h) dst[h] = 0;
+    }
+    if (r == kB3BlockGroups - 1)
+      *reinterpret_cast<uint2*>(stage + (lane / kB3BlockGroups) * kB3BlockBytes + kB3GroupBytes * kB3BlockGroups) =
+          make_uint2(0u, 0u);
+    __syncwarp();
+    // The run's whole blocks (all 8 but at the very end), 16 bytes a thread.
+    const int64_t left = (total - base) / kB3BlockGroups;
+    const int chunks = (left < kWarpBlocks ? static_cast<int>(left) : kWarpBlocks) * (kB3BlockBytes / 16);
+    uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(packed) + base / kB3BlockGroups * kB3BlockBytes);
+    for (int c16 = lane; c16 < chunks; c16 += 32) out[c16] = reinterpret_cast<const uint4*>(stage)[c16];
+    __syncwarp();
   }
   if (!__all_sync(0xffffffffu, ok) && lane_id() == 0) atomicOr(&g_pack_bad_code, 1u);
 }

@@ -461,6 +461,21 @@ __host__ __device__ constexpr uint32_t f16_instr_desc(int m, int n) {
   return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// ------------------------------------------------------- global loads ---
+// One 32-byte read-only load (the address 32-byte aligned) as two uint4.
+__device__ __forceinline__ void ldg_32b(const void* p, uint4& lo, uint4& hi) {
+  asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+               : "l"(reinterpret_cast<uint64_t>(p)));
+}
+
+// One 32-byte store (the address 32-byte aligned) of two uint4.
+__device__ __forceinline__ void stg_32b(void* p, const uint4& lo, const uint4& hi) {
+  asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+               : "memory");
+}
+
 // ------------------------------------------------------------ bit ops ---
 // (a & b) | c in one three-input logic instruction, b and c in registers.
 __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {

@@ -84,6 +84,18 @@ def test_pack_bit_exact(oracle_mod, mode, N, K):
     assert np.array_equal(to_u32(got), ref)
 
 
+@pytest.mark.parametrize("mode", MODES)
+def test_pack_bit_exact_from_16_byte_aligned_codes(oracle_mod, mode):
+    """Codes that are 16- but not 32-byte aligned take the 16-byte load path."""
+    d = workloads.make(mode=mode, M=1, N=129, K=1152, seed=99)
+    buf = torch.empty(d["codes"].size + 16, dtype=torch.int8, device="cuda")
+    assert buf.data_ptr() % 32 == 0
+    codes = buf[16:].view(129, 1152)
+    codes.copy_(dev(d["codes"]))
+    assert codes.data_ptr() % 32 == 16
+    assert np.array_equal(to_u32(bw.pack(codes, mode)), oracle_mod.pack(d["codes"], mode))
+
+
 @pytest.mark.parametrize("mode,bad", [("ternary", 2), ("ternary", -2), ("binary", 0), ("binary", 3),
                                       ("ternary_b3", 2), ("ternary_b3", -128)])
 def test_pack_reports_bad_codes(mode, bad):
@@ -105,6 +117,20 @@ def test_dequant_bit_exact(oracle_mod, mode, N, K):
     ref = oracle_mod.dequant(ref_packed, d["scales"], K, mode)
     got = bw.dequant(packed, scales, K, mode)
     assert np.all(nan_aware_equal(to_u16(got), ref))
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_dequant_bit_exact_into_16_byte_aligned_output(oracle_mod, mode):
+    """An output 16- but not 32-byte aligned takes the 16-byte store path."""
+    N, K = 129, 1152
+    d = workloads.make(mode=mode, M=1, N=N, K=K, seed=98)
+    ref_packed, packed, _, scales = gpu_inputs(d, oracle_mod)
+    buf = torch.empty(N * K + 8, dtype=torch.float16, device="cuda")
+    assert buf.data_ptr() % 32 == 0
+    out = buf[8:].view(N, K)
+    assert out.data_ptr() % 32 == 16
+    bw.dequant(packed, scales, K, mode, out=out)
+    assert np.all(nan_aware_equal(to_u16(out), oracle_mod.dequant(ref_packed, d["scales"], K, mode)))
 
 
 @pytest.mark.parametrize("mode", MODES)
