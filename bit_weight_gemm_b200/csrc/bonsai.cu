@@ -258,12 +258,13 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, c
   if (smem_opt_in<lowbit_gemm_kernel<MODE, BLOCK_T>>(T::kSmemBytes) != BONSAI_OK) return BONSAI_ERR_CUDA;
 
   CUtensorMap map_act, map_w, map_out;
-  if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, BLOCK_T, CU_TENSOR_MAP_SWIZZLE_128B))
+  // Boxes of one MMA's tokens (half of a two-half tile).
+  if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, K, M, 64, T::kMmaN, CU_TENSOR_MAP_SWIZZLE_128B))
     return BONSAI_ERR_CUDA;
   if (!make_weight_map(&map_w, packed, N, K, MODE)) return BONSAI_ERR_CUDA;
   const bool tma_store = (N % 8) == 0;
   if (tma_store) {
-    if (!make_map(&map_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, out, N, M, T::kRows, BLOCK_T,
+    if (!make_map(&map_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, out, N, M, T::kRows, T::kMmaN,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
       return BONSAI_ERR_CUDA;
   } else {
@@ -271,7 +272,7 @@ int launch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales, c
   }
   const int groups = K / kGroup;
   const int tiles_n = (N + T::kRows - 1) / T::kRows, tiles_m = (M + BLOCK_T - 1) / BLOCK_T;
-  if (ksplit < 1 || ksplit > 8 || ksplit > groups) return BONSAI_ERR_SHAPE;
+  if (ksplit < 1 || ksplit > 8 || ksplit > groups || (T::kHalves > 1 && ksplit > 1)) return BONSAI_ERR_SHAPE;
   // Scale tile by TMA: rows of the scale matrix must be 16-byte multiples
   // (groups % 8 == 0); the box covers a CTA's groups from an 8-aligned start.
   CUtensorMap map_s = map_act;  // placeholder when unused
@@ -565,7 +566,8 @@ constexpr TileCost tile_cost(int block_t) {
          : block_t == 128 ? TileCost{0.50, 2.5, 2.0}
          : block_t == 176 ? TileCost{0.59, 2.7, 2.75}  // interpolated between 128 and 192
          : block_t == 192 ? TileCost{0.62, 2.75, 3.0}
-                          : TileCost{0.75, 3.0, 4.0};
+         : block_t == 256 ? TileCost{0.75, 3.0, 4.0}
+                          : TileCost{1.12, 3.5, 0.0};  // 352 (two halves; not split), measured at 2048 tokens
 }
 constexpr double kLaunchCost = 2.5;
 constexpr double kPersistentBoundary = 1.0;
@@ -588,6 +590,9 @@ void consider(int M, int N, int K, Plan* best) {
   // Base-3 ranges start on 4-group blocks: at most groups / 4 of them.
   const int max_ks = MODE == BONSAI_TERNARY_B3 ? (groups / kB3BlockGroups > 1 ? groups / kB3BlockGroups : 1) : groups;
   for (int ks = 1; ks <= 8 && ks <= max_ks; ++ks) {
+    if constexpr (BLOCK_T > 256) {
+      if (ks > 1) break;  // two-half tiles are not split
+    }
     const int per_wave = ks == 1 ? sms : resident_clusters<MODE, BLOCK_T>(ks);
     if (per_wave <= 0) continue;
     const int waves = (tiles + per_wave - 1) / per_wave;
@@ -595,8 +600,13 @@ void consider(int M, int N, int K, Plan* best) {
     // layers); with more tiles the persistent 192- or 256-token forms win
     // (measured at 2048 tokens, N=3072, K=9216: 1068 TFLOP/s against ~1300).
     if (BLOCK_T == 176 && waves > 1) continue;
+    // 352-token tiles (two 176-token halves) likewise, and unsplit: at 2048
+    // tokens the N=3072 layers make 144 of them, one wave, where 192-token
+    // tiles need 1.8 waves of the persistent kernel; on ragged mid-M shapes
+    // just past one wave of 256-token tiles they save a second wave.
+    if (BLOCK_T == 352 && waves > 1) continue;
     bool persistent = false;
-    if constexpr (BLOCK_T >= 192) persistent = ks == 1 && use_persistent<MODE, BLOCK_T>(M, N, K);
+    if constexpr (BLOCK_T >= 192 && BLOCK_T <= 256) persistent = ks == 1 && use_persistent<MODE, BLOCK_T>(M, N, K);
     const double per_wave_cost = ((groups + ks - 1) / ks) * c.group + (persistent ? kPersistentBoundary : c.wave) +
                                  (ks > 1 ? c.reduce : 0.0);
     const double cost = kLaunchCost + waves * per_wave_cost;
@@ -641,6 +651,9 @@ Plan plan_gemm(int M, int N, int K) {
     consider<MODE, 176>(M, N, K, &best);
     consider<MODE, 192>(M, N, K, &best);
     consider<MODE, 256>(M, N, K, &best);
+    // Ternary weights only: binary ones measured 6% slower in 352-token tiles
+    // than in the persistent kernel's 192-token tiles at 2048 tokens.
+    if constexpr (MODE == BONSAI_TERNARY_INT2 || MODE == BONSAI_TERNARY_B3) consider<MODE, 352>(M, N, K, &best);
   }
   return best;
 }
@@ -663,6 +676,10 @@ int dispatch_gemm(const uint16_t* A, const void* packed, const uint16_t* scales,
     case 176: return launch_gemm<MODE, 176>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 192: return launch_gemm<MODE, 192>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
     case 256: return launch_gemm<MODE, 256>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+    case 352:
+      if constexpr (MODE == BONSAI_TERNARY_INT2 || MODE == BONSAI_TERNARY_B3)
+        return launch_gemm<MODE, 352>(A, packed, scales, zeros, M, N, K, p.ksplit, out, stream);
+      return BONSAI_ERR_CUDA;
     default: return BONSAI_ERR_CUDA;  // no plan: the occupancy queries failed
   }
 }

@@ -79,10 +79,18 @@ struct GemmTile {
   static constexpr int kWordsPerGroup = MODE == BONSAI_BINARY ? 4 : (kB3 ? 7 : (kHqq ? 16 : 8));
   static constexpr int kSliceBytes = BLOCK_T * 128;       // BLOCK_T rows x 64 FP16
   static constexpr int kActStageBytes = 2 * kSliceBytes;  // 128 K per stage
+  // Tiles wider than one MMA (352 tokens) run as two halves of kMmaN tokens:
+  // two MMAs per K step into two accumulators (the second at TMEM column
+  // kHalfCol, 64-aligned), and TMA boxes of kMmaN rows (a box has at most
+  // 256).
+  static constexpr int kHalves = BLOCK_T > 256 ? 2 : 1;
+  static constexpr int kMmaN = BLOCK_T / kHalves;
+  static constexpr int kHalfCol = kHalves == 2 ? (kMmaN + 63) / 64 * 64 : 0;
+  static constexpr int kHalfBytes = kMmaN * 128;  // one half of a K slice
   // Activation stages: as many as fit next to the word ring and the scales,
   // so that narrow tiles keep a split-K CTA's whole K range in flight.
   static constexpr int kActStages =
-      BLOCK_T > 128 ? 3 : (BLOCK_T == 128 ? 4 : (96 * 1024) / kActStageBytes);
+      BLOCK_T > 256 ? 2 : (BLOCK_T > 128 ? 3 : (BLOCK_T == 128 ? 4 : (96 * 1024) / kActStageBytes));
   // A word stage is 128 bytes of every row: 4 ternary or 8 binary groups,
   // one TMA box with 128-byte swizzling.
   // Base-3: one 112-byte block (4 groups) of every row per stage, without
@@ -100,8 +108,10 @@ struct GemmTile {
   // (4-bit group-affine weights keep scale and zero pairs in registers.)
   static constexpr int kScaleBytes = (BLOCK_T >= 256 || kHqq) ? 0 : 32768;
   // Converter warps: four per TMEM lane quadrant.  (Five per quadrant on
-  // narrow tiles measured 2-5% slower.)
-  static constexpr int kConvWarps = 16;
+  // narrow tiles measured 2-5% slower.)  Two-half tiles leave room for two
+  // TMEM stages only, and a quadrant may have no more warps than stages
+  // (below); a group is then ~1400 cycles of MMAs, ample for two.
+  static constexpr int kConvWarps = kHalves == 2 ? 8 : 16;
   static constexpr int kWarpsPerQuad = kConvWarps / 4;
   // Epilogue: the quadrant's warps split the token columns, 8 at least each:
   // the most warps (up to kWarpsPerQuad) that divide BLOCK_T / 8.
@@ -118,7 +128,8 @@ struct GemmTile {
   // with narrow tiles an MMA is a few cycles of work, so a chain of MMAs into
   // one accumulator would run at the accumulate latency instead.
   static constexpr int kAccs = (kMmaThreads == 2 || BLOCK_T <= 32) ? 2 : 1;
-  static constexpr int kACol0 = kAccs * BLOCK_T < 64 ? 64 : kAccs * BLOCK_T;  // converted-weight stages follow
+  static constexpr int kACol0 = kHalves == 2 ? 2 * kHalfCol
+                                : (kAccs * BLOCK_T < 64 ? 64 : kAccs * BLOCK_T);  // converted-weight stages follow
   // TMEM stages of converted weights, 64 columns each: all that is left
   // after the accumulators.  A stage is reused only after the MMAs that read
   // it completed, so the number of stages is the number of groups in flight
@@ -141,7 +152,8 @@ struct GemmTile {
   static constexpr int kSmemBytes = kSmemNeeded < 116 * 1024 ? 116 * 1024 : kSmemNeeded;
 
   static constexpr float kOutScale = MODE == BONSAI_TERNARY_INT2 ? 0.5f : 1.0f;  // INT2 converts to 2ts
-  static_assert(BLOCK_T % 16 == 0 && BLOCK_T >= 16 && BLOCK_T <= 256, "MMA N for M=128");
+  static_assert(kMmaN % 16 == 0 && kMmaN >= 16 && kMmaN <= 256 && kMmaN * kHalves == BLOCK_T, "MMA N for M=128");
+  static_assert(kHalves == 1 || (kAccs == 1 && kHalfCol >= kMmaN && kHalfBytes % 1024 == 0), "two-half tiles");
   static_assert(kSliceBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kACol0 + kTStages * 64 <= kTmemCols && kTStages >= 2, "TMEM budget");
   // Parity waits on a TMEM stage are unambiguous only if the converter is at
@@ -395,8 +407,11 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       mbar_arrive_expect_tx_elected(full, T::kActStageBytes);
       const uint32_t dst = smem_addr(smem + T::kActOff + s * T::kActStageBytes);
       const int k = (g_begin + i) * kGroup;
-      tma_load_2d_elected(dst, &tmap_act, full, k, m0);
-      tma_load_2d_elected(dst + T::kSliceBytes, &tmap_act, full, k + 64, m0);
+#pragma unroll
+      for (int h = 0; h < T::kHalves; ++h) {  // rows m0 + h * kMmaN .. of each K slice
+        tma_load_2d_elected(dst + h * T::kHalfBytes, &tmap_act, full, k, m0 + h * T::kMmaN);
+        tma_load_2d_elected(dst + T::kSliceBytes + h * T::kHalfBytes, &tmap_act, full, k + 64, m0 + h * T::kMmaN);
+      }
       issued = i + 1;
     }
     if (*abort_flag) {  // let copies in flight land before the CTA's memory goes away
@@ -443,7 +458,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     constexpr int kOwnAccs = T::kAccs / P;  // accumulators per issuing warp
     const int first = warp == 1 ? 0 : 1;
     if (first < P) {
-      constexpr uint32_t idesc = f16_instr_desc(128, BLOCK_T);
+      constexpr uint32_t idesc = f16_instr_desc(128, T::kMmaN);
       // Descriptor of act stage 0; other stages and K steps add their byte
       // offset >> 4 to the start-address field (no carry: shared memory
       // addresses stay below 256 KB).
@@ -460,7 +475,11 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = desc_s + static_cast<uint64_t>(((kk >> 2) * T::kSliceBytes + (kk & 3) * 32) >> 4);
           const int acc = (step % kOwnAccs) * P + first;
-          mma_f16_tmem_a_elected(tmem + acc * BLOCK_T, a_cols + kk * 8, bdesc, idesc, step >= kOwnAccs ? 1u : 0u);
+#pragma unroll
+          for (int h = 0; h < T::kHalves; ++h)  // half h: tokens h * kMmaN .., accumulator at column h * kHalfCol
+            mma_f16_tmem_a_elected(tmem + acc * BLOCK_T + h * T::kHalfCol, a_cols + kk * 8,
+                                   bdesc + static_cast<uint64_t>((h * T::kHalfBytes) >> 4), idesc,
+                                   step >= kOwnAccs ? 1u : 0u);
           ++step;
         }
         mma_commit_elected(act_empty0 + 8 * sa);
@@ -610,6 +629,8 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
     const int used_accs = (T::kMmaThreads == 2 && ng < 2) ? 1 : T::kAccs;
     const bool epi = turn < T::kEpiWarpsPerQuad;
     const int c_begin = turn * kEpiCols;
+    // TMEM column of token column c (8-column runs never straddle the halves).
+    auto acc_col = [](int c) { return c < T::kMmaN ? c : c - T::kMmaN + T::kHalfCol; };
     if (args.ksplit == 1) {
       // FP16 tile [BLOCK_T tokens][128 rows] in the (now idle) act ring.
       uint16_t* tile = reinterpret_cast<uint16_t*>(smem + T::kActOff);
@@ -617,7 +638,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < kEpiCols; c += 8) {
           float acc[8];
-          sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, used_accs, acc);
+          sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + acc_col(c_begin + c), used_accs, acc);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const __half h = __float2half_rn(acc[j] * T::kOutScale);
@@ -630,7 +651,12 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
       if (*abort_flag == 0) {
         if (args.tma_store) {
           if (warp == 3 && lane == 0) {
-            tma_store_2d(&tmap_out, smem_addr(tile), n0, m0);
+            // Halves that start past the last token are not stored (a store
+            // box starts inside the tensor).
+#pragma unroll
+            for (int h = 0; h < T::kHalves; ++h)
+              if (h == 0 || m0 + h * T::kMmaN < args.M)
+                tma_store_2d(&tmap_out, smem_addr(tile) + h * T::kMmaN * T::kRows * 2, n0, m0 + h * T::kMmaN);
             bulk_commit_group();
             bulk_wait_group_read0();
           }
@@ -648,7 +674,7 @@ __global__ void __launch_bounds__(GemmTile<MODE, BLOCK_T>::kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < kEpiCols; c += 8) {
         float acc[8];
-        sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + c_begin + c, used_accs, acc);
+        sum_accumulators<T::kAccs, BLOCK_T>(tmem + lane_base + acc_col(c_begin + c), used_accs, acc);
 #pragma unroll
         for (int j = 0; j < 8; ++j) part[(c_begin + c + j) * T::kRows + row] = acc[j];
       }

@@ -256,16 +256,17 @@ def test_plan_in_a_fresh_process_matches_launch():
 # Large M: more tiles than SMs.  With K a multiple of 512 (ternary) or 1024
 # (binary) one persistent CTA per SM walks the 256-token tiles; else each
 # 128- or 256-token tile is its own CTA over several waves.  Ragged M and N;
-# 186, 150 and 237 tiles leave persistent CTAs with one and with two tiles;
-# N odd in the third case.
+# 234, 225 and 237 tiles leave persistent CTAs with one and with two tiles;
+# N odd in the fifth case.  (N is wide enough that 352-token tiles would not
+# fit one wave, so these shapes keep the forms they test.)
 LARGE_M_SHAPES = [
-    ("ternary", 1357, 3880, 512, True),
-    ("ternary_b3", 1357, 3880, 512, True),
-    ("ternary_b3", 700, 6376, 1152, False),
-    ("binary", 700, 6376, 1024, True),
+    ("ternary", 1357, 4990, 512, True),
+    ("ternary_b3", 1357, 4990, 512, True),
+    ("ternary_b3", 700, 9600, 1152, False),
+    ("binary", 700, 9600, 1024, True),
     ("ternary", 513, 9999, 1024, True),
-    ("ternary", 1357, 3880, 640, False),
-    ("binary", 600, 6376, 512, False),
+    ("ternary", 1357, 4990, 640, False),
+    ("binary", 600, 9600, 512, False),
 ]
 
 
@@ -279,9 +280,15 @@ MID_M_TILE_SHAPES = [
     ("ternary", 1000, 3000, 1152, 176, False),
     ("ternary_b3", 1000, 3000, 1152, 176, False),
     ("ternary", 1024, 3072, 12288, 176, False),
-    ("ternary", 2048, 3072, 2048, 192, True),
-    ("ternary_b3", 2000, 3050, 2048, 192, True),
-    ("binary", 2048, 3072, 2048, 192, True),
+    ("ternary", 2304, 3072, 2048, 192, True),
+    ("ternary_b3", 2300, 3050, 2048, 192, True),
+    ("binary", 2304, 3072, 2048, 192, True),
+    # 352-token tiles (two 176-token halves, ternary formats): 144 one-wave CTAs at ~2048 tokens on N ~ 3072
+    ("ternary", 2048, 3072, 2048, 352, False),
+    ("ternary_b3", 2000, 3050, 2048, 352, False),
+    ("ternary", 1800, 3072, 2048, 352, False),  # the last tile's second half starts past M: not stored
+    ("ternary", 2048, 2996, 1152, 352, False),  # N % 8 != 0: direct stores instead of TMA
+    ("ternary_b3", 700, 6376, 1152, 352, False),  # 100 tiles, where 256-token ones make 150 (two waves)
 ]
 
 
