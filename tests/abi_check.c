@@ -43,6 +43,24 @@ int main(void) {
   expect(bonsai_lowbit_gemm_batch(batch, 1, BONSAI_TERNARY_INT2, NULL), BONSAI_ERR_SHAPE, "batch: K % 128");
   expect(bonsai_lowbit_gemm_batch(batch, -1, BONSAI_TERNARY_INT2, NULL), BONSAI_ERR_INVALID_ARG, "batch: count");
   expect(bonsai_lowbit_gemm_batch(NULL, 0, BONSAI_TERNARY_INT2, NULL), BONSAI_OK, "batch: empty");
+  expect(bonsai_lowbit_gemm_batch(NULL, 2, BONSAI_TERNARY_INT2, NULL), BONSAI_ERR_INVALID_ARG, "batch: null list");
+  expect(bonsai_lowbit_gemm_batch(batch, 1, 7, NULL), BONSAI_ERR_INVALID_ARG, "batch: mode");
+  batch[0].K = 128; /* shapes fine, output missing */
+  expect(bonsai_lowbit_gemm_batch(batch, 1, BONSAI_BINARY, NULL), BONSAI_ERR_INVALID_ARG, "batch: null out");
+  batch[0].M = 0; /* an empty problem needs no buffers */
+  expect(bonsai_lowbit_gemm_batch(batch, 1, BONSAI_BINARY, NULL), BONSAI_OK, "batch: only empty problems");
+
+  /* 4-bit group-affine weights: half a byte per weight, same argument rules */
+  expect((int)(bonsai_hqq4_packed_bytes(3072, 9216) == (size_t)3072 * 9216 / 2), 1, "4-bit bytes");
+  expect(bonsai_hqq4_pack(NULL, 4, 100, NULL, NULL), BONSAI_ERR_SHAPE, "4-bit pack: K % 128");
+  expect(bonsai_hqq4_pack(NULL, 4, 128, NULL, NULL), BONSAI_ERR_INVALID_ARG, "4-bit pack: null");
+  expect(bonsai_hqq4_gemm(NULL, NULL, NULL, NULL, 4, 4, 128, NULL, NULL), BONSAI_ERR_INVALID_ARG, "4-bit gemm: null");
+
+  /* plan query: an empty GEMM plans nothing and needs no device */
+  int bt = -1, ks = -1, ctas = -1, tiles = -1;
+  expect(bonsai_gemm_plan(0, 8, 128, BONSAI_BINARY, &bt, &ks, &ctas, &tiles), BONSAI_OK, "plan: empty");
+  expect(bt | ks | ctas | tiles, 0, "plan: empty is all zeros");
+  expect(bonsai_gemm_plan(4, 8, 100, BONSAI_BINARY, &bt, &ks, &ctas, &tiles), BONSAI_ERR_SHAPE, "plan: K % 128");
 
   if (failures) return 1;
   printf("ok\n");
