@@ -116,11 +116,12 @@ def test_batch_with_empty_and_k0_problems(oracle_mod):
     check_all(oracle_mod, mode, probs, [outs[0], outs[3]], "batch with empty problems")
 
 
-def test_batch_larger_than_one_launch(oracle_mod):
-    """100 problems: more than one persistent launch takes, so two launches."""
-    mode = "ternary"
+@pytest.mark.parametrize("mode", MODES)
+def test_batch_larger_than_one_launch(oracle_mod, mode):
+    """100 problems: more than one persistent launch takes, so two launches;
+    1 to 5 groups per row, so word stages both whole and ragged."""
     shapes = [(1 + j % 16, 8 * (1 + j % 40), 128 * (1 + j % 5)) for j in range(100)]
-    probs = build(oracle_mod, mode, shapes, 7200)
+    probs = build(oracle_mod, mode, shapes, 7200 + MODES.index(mode))
     outs = bw.lowbit_gemm_batch([(p["A"], p["packed"], p["s"]) for p in probs], mode)
     torch.cuda.synchronize()
     check_all(oracle_mod, mode, probs, outs, "100-problem batch")
